@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP4 W4A4 linear layer on B200: quantize activations + block-scaled GEMM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxq|reference] [--workload NAME]
+
+One step = one mxq_linear call over one batch of the prefill gate+up problem
+(A [8192, 5120] bf16 -> MXFP4 CEIL per token, W [34816, 5120] pre-quantized MXFP4 EVEN, bf16 out):
+dynamic activation quantization (block amax, scale, encode, pack, swizzled scales) and the
+tcgen05 GEMM with its bf16 epilogue.  The metric is 2*M*N*K / step time, in TFLOP/s.
+
+Per rank the working set (A 84 MB + W 95 MB read, 570 MB written per step) is larger than the
+126 MB L2, so no separate L2 flush is done between steps.  Under torchrun every rank runs its own
+copy of the problem (weak scaling, no collective on the data path); the timed region is bracketed
+by a barrier + synchronize and the max over ranks is reported.
+
+`--impl reference` times the scalar CPU oracle (quantize + fp64 GEMM) on a bounded sample of the
+same problem on the host cores, in the same unit.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from nvfp4_block_scaled_mx_b200 import synth  # noqa: E402
+
+METRIC = "MXFP4 W4A4 linear TFLOPS (act-quant+GEMM) and quantize GB/s vs B200 peaks"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+FP4_PER_BF16 = 4.0   # nominal dense fp4 : bf16 tensor throughput (9 : 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0
+# algorithmic bytes per element of the quantizer: 2 B read + elements written + scale bytes
+QUANT_BYTES_PER_ELEM = {"mxfp4": 2.0 + 0.5 + 1 / 32, "nvfp4": 2.0 + 0.5 + 1 / 16, "mxfp8": 2.0 + 1.0 + 1 / 32}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
+    ap.add_argument("--workload", default="prefill_gate_up")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def traffic_for(key):
+    if os.path.exists(TRAFFIC_PATH):
+        with open(TRAFFIC_PATH) as fh:
+            return json.load(fh).get(key)
+    return None
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_weak(per_rank_units, world):
+    """Whole-job units: every rank processes the same per-rank amount (weak scaling)."""
+    return per_rank_units * world
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        # the timed region is the busy part of the sampling window: report the upper half
+        busy = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- the mxq arm
+
+def time_loop(fn, iters, stream):
+    """Average device time of fn() over iters launches, CUDA events on `stream`."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(iters):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / iters / 1e3
+
+
+def run_mxq(args, world, rank, local):
+    from nvfp4_block_scaled_mx_b200 import mxq
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl mxq needs a CUDA device (there is no CPU fallback)")
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.workload]
+    M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
+    stream = torch.cuda.current_stream(dev)
+    hbm_gbs, bf16_tflops, peak_src = peaks()
+
+    A, W = synth.make_inputs(args.workload, device=dev)
+    g_w = g_a = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(W)
+        g_a, _ = mxq.global_scale(A)
+    W_q, W_sf = mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED)
+    ws = torch.empty(mxq.mxq_linear_workspace_size(M, K, mxq.FMT[fmt]), dtype=torch.uint8, device=dev)
+    out_dtype = torch.float32 if cfg["out"] == "fp32" else torch.bfloat16
+    out = torch.empty(M, N, dtype=out_dtype, device=dev)
+    flops = 2.0 * M * N * K
+
+    def step():
+        mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
+                   workspace=ws, out=out, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    mxq.mxq_device_status(reset=True)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed = start.elapsed_time(end) / 1e3
+    status = mxq.mxq_device_status(reset=True)
+    if status != 0:
+        raise SystemExit("a kernel reported a bounded-wait timeout (status 0x%x)" % status)
+    elapsed_max = max_over_ranks(elapsed, world, dev)
+    value = aggregate_weak(flops * args.steps, world) / elapsed_max / 1e12
+
+    # dominant kernel timed alone: the GEMM on the step's own quantized activations
+    a_q = ws[: M * K // 2].view(M, K // 2) if fmt != "mxfp8" else ws[: M * K].view(M, K)
+    qbytes = a_q.numel()
+    a_sf = ws[(qbytes + 255) // 256 * 256:]
+    gemm_s = time_loop(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a, g_B=g_w,
+                                        out=out, stream=stream), max(10, args.steps // 4), stream)
+    quant_s = time_loop(lambda: mxq.quantize(A, fmt, cfg["a_rule"], global_scale=g_a, layout=mxq.SF_SWIZZLED,
+                                             q_out=a_q, sf_out=a_sf, stream=stream), max(10, args.steps // 4), stream)
+    tensor_peak = bf16_tflops * (FP8_PER_BF16 if fmt == "mxfp8" else FP4_PER_BF16)
+    gemm_tflops = flops / gemm_s / 1e12
+    roofline = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::%s)" % {"mxfp4": "mxf4", "nvfp4": "mxf4nvf4",
+                                                                                 "mxfp8": "mxf8f6f4"}[fmt],
+                "achieved": round(gemm_tflops, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+                "frac": round(gemm_tflops / tensor_peak, 4),
+                "peak_source": "%s bf16 %.1f TFLOP/s x %g nominal %s:bf16 ratio" % (
+                    peak_src, bf16_tflops, FP4_PER_BF16 if fmt != "mxfp8" else FP8_PER_BF16, fmt),
+                "frac_of_datasheet": round(gemm_tflops / (9000.0 if fmt != "mxfp8" else 4500.0), 4),
+                "traffic": traffic_for("gemm_%s_%s" % (fmt, args.workload)),
+                "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
+    qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
+    quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
+             "gbs": round(qb / quant_s / 1e9, 1), "frac": round(qb / quant_s / 1e9 / hbm_gbs, 4),
+             "peak_gbs": hbm_gbs, "ms": round(quant_s * 1e3, 4), "algorithmic_bytes": qb}
+
+    # weight (RTN, EVEN) quantizer on the 451 MB weight tensor
+    wq_s = time_loop(lambda: mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED, q_out=W_q,
+                                          sf_out=W_sf, stream=stream), 20, stream)
+    wb = QUANT_BYTES_PER_ELEM[fmt] * N * K
+    quant_w = {"workload": "weight quantize %dx%d %s %s" % (N, K, fmt, cfg["w_rule"]),
+               "gbs": round(wb / wq_s / 1e9, 1), "frac": round(wb / wq_s / 1e9 / hbm_gbs, 4), "peak_gbs": hbm_gbs,
+               "ms": round(wq_s * 1e3, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(step, A, out, flops, args, stream, world, dev)
+
+    res = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "e2m1xe2m1->f32 (bf16 out)" if fmt != "mxfp8" else
+           "e4m3xe4m3->f32 (bf16 out)", "data": "synthetic (seeded, random-init weights)",
+           "config": {"workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt, "act_rule": cfg["a_rule"],
+                      "weight_rule": cfg["w_rule"], "out": cfg["out"], "l2": "working set > 126 MB L2, no flush",
+                      "parallelism": "replicas x%d (no collective)" % world},
+           "gpu_launches": 2 * args.steps, "roofline": roofline, "quantize": quant, "quantize_weight": quant_w,
+           "clocks": clk.summary(), "e2e": e2e}
+    return res
+
+
+def run_e2e(step, A, out, flops, args, stream, world, dev):
+    """Same step through host buffers: pinned H2D of A, the linear, D2H of the output."""
+    A_h = torch.empty(A.shape, dtype=A.dtype, pin_memory=True)
+    A_h.copy_(A)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    iters = max(3, min(20, args.steps // 10))
+
+    def e2e_step():
+        A.copy_(A_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t = time_loop(e2e_step, iters, stream)
+    t = max_over_ranks(t, world, dev)
+    return {"value": round(aggregate_weak(flops, world) / t / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": A.numel() * A.element_size(), "d2h_bytes_per_step": out.numel() * out.element_size(),
+            "ms_per_step": round(t * 1e3, 3)}
+
+
+# ---------------------------------------------------------------- the oracle (CPU) arm
+
+def oracle_sample(workload, rows, cols, seed=0):
+    """Inputs of a bounded CPU sample: `rows` activation rows and `cols` weight rows of the problem."""
+    cfg = synth.CONFIGS[workload]
+    gen = synth.make_generator(1000 * cfg["seed"] + 7 + seed)
+    A = synth.draw_matrix(rows, cfg["K"], cfg["a"], gen)
+    W = synth.draw_matrix(cols, cfg["K"], cfg["w"], gen)
+    return cfg, A, W
+
+
+def oracle_step(orc, cfg, A, Wq, Wsf, gW):
+    fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
+    rules = {"even": orc.EVEN, "ceil": orc.CEIL}
+    f = fmts[cfg["fmt"]]
+    gA = 1.0
+    if cfg["fmt"] == "nvfp4":
+        gA, _ = orc.global_scale(A)
+    Aq, Asf = orc.quantize(A, f, rules[cfg["a_rule"]], g=float(gA))
+    orc.gemm(Aq, Asf, Wq, Wsf, A.shape[0], Wq.shape[0], cfg["K"], f, gA=float(gA), gB=float(gW))
+
+
+def cpu_baseline(workload, rows=256, cols=4096):
+    import oracle as orc
+    cfg, A, W = oracle_sample(workload, rows, cols)
+    fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
+    rules = {"even": orc.EVEN, "ceil": orc.CEIL}
+    gW = 1.0
+    if cfg["fmt"] == "nvfp4":
+        gW, _ = orc.global_scale(W)
+    Wq, Wsf = orc.quantize(W, fmts[cfg["fmt"]], rules[cfg["w_rule"]], g=float(gW))
+    t0 = time.perf_counter()
+    oracle_step(orc, cfg, A, Wq, Wsf, gW)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * cols * cfg["K"]
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": "%d activation rows x %d weight rows x K=%d of %s: CEIL/EVEN quantize of the rows + fp64 "
+                      "GEMM, single-threaded scalar C, %.1f s" % (rows, cols, cfg["K"], workload, dt)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle as orc
+    orc.build()
+    rows, cols = 8, 512
+    cfg, A, W = oracle_sample(args.workload, rows, cols)
+    fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
+    rules = {"even": orc.EVEN, "ceil": orc.CEIL}
+    gW = 1.0
+    if cfg["fmt"] == "nvfp4":
+        gW, _ = orc.global_scale(W)
+    Wq, Wsf = orc.quantize(W, fmts[cfg["fmt"]], rules[cfg["w_rule"]], g=float(gW))
+    for _ in range(max(1, args.warmup)):
+        oracle_step(orc, cfg, A, Wq, Wsf, gW)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(orc, cfg, A, Wq, Wsf, gW)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * cols * cfg["K"]
+    value = flops * args.steps / dt / 1e12
+    sample = ("per step %d activation rows x %d weight rows x K=%d of %s (quantize rows + fp64 GEMM), "
+              "scalar C oracle, 1 thread" % (rows, cols, cfg["K"], args.workload))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": args.workload, "M": cfg["M"], "N": cfg["N"],
+                                                     "K": cfg["K"], "fmt": cfg["fmt"]},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_mxq(args, world, rank, local)
+            if rank == 0 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(args.workload)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

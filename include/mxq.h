@@ -1,0 +1,140 @@
+/*
+ * mxq.h -- C ABI of the B200 (sm_100a) microscaling W4A4 linear-layer library (libmxq.so).
+ *
+ * The library implements the hot path of a block-scaled quantized linear layer,
+ * Out = A * W^T with A [M, K] activations and W [N, K] weights (nn.Linear layout):
+ *   - MXFP4: E2M1 elements in blocks of 32 along K with one E8M0 (power-of-two) scale per block,
+ *     the EVEN rule for weights and the CEIL rule for per-token dynamic activation quantization
+ *     ("Qwen3.5-27B-MXFP4-QAD-W4A4-LR1e-5-s1000", "How this checkpoint was produced", Training row;
+ *      "Qwen3.5-9B-MXFP4-QAD-W4A4-LR1e-5-s3000", "Training mode" paragraph);
+ *   - NVFP4: E2M1 elements, blocks of 16 with an E4M3 scale, and one fp32 per-tensor global scale
+ *     ("Qwen3.5-27B-NVFP4-RTN-weight-only", first paragraph; "Qwen3.5-27B-NVFP4-GPTQ", Recipe row);
+ *   - MXFP8: E4M3 elements, blocks of 32 with an E8M0 scale
+ *     ("intel-ai/Qwen3.8-27B-MXFP4-AutoRound", section 1 and section 7, OCP MX).
+ *
+ * Scale rules (block amax over |x|, e clamped to [-127, 127], amax = 0 gives e = -127):
+ *   EVEN  e = floor(log2 amax) - emax_elem           (emax_elem 2 for E2M1, 8 for E4M3)
+ *   CEIL  e = least integer with amax <= elem_max * 2^e   (elem_max 6 for E2M1, 448 for E4M3)
+ * MX elements are RNE(x / 2^e) on the element grid, saturating at +-elem_max.
+ * NVFP4 (fp32 IEEE, g = global scale in the decode direction, x ~ q * s * g):
+ *   s = RNE_E4M3_satfinite(fl(fl(amax/6) / g)) (0 for an all-zero block), d = fl(dec(s) * g),
+ *   q_i = RNE_E2M1_sat(fl(x_i * fl(1/d))); when d == 0 every code is a zero that keeps x_i's sign.
+ *
+ * Conventions for every call:
+ *   - Pointers marked (device) are device memory of the current CUDA device; the caller owns and
+ *     allocates every buffer.  The compute calls allocate nothing.
+ *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Return MXQ_OK (0) or a negative MXQ_ERR_* code.  Argument errors are detected on the host
+ *     before anything is launched; MXQ_ERR_CUDA reports a failed launch.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Quantized FP4 data: [rows, K/2] bytes, element 2i in bits 0-3 and element 2i+1 in bits 4-7
+ *     of byte i of the row.  MXFP8 data: [rows, K] bytes of E4M3 codes.
+ *   - Row-major scales: [rows, K/bs] bytes.  Swizzled scales (what the GEMM consumes): tiles of
+ *     128 rows x 4 scale columns, 512 bytes each, ordered [ceil(rows/128)][ceil((K/bs)/4)]; inside a
+ *     tile, scale (r, c) sits at byte (r%32)*16 + ((r%128)/32)*4 + c%4.  Padding bytes are zero.
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mxq_stream_t; /* same type as cudaStream_t */
+
+typedef enum { MXQ_MXFP4 = 0, MXQ_NVFP4 = 1, MXQ_MXFP8 = 2 } mxq_fmt;
+typedef enum { MXQ_RULE_EVEN = 0, MXQ_RULE_CEIL = 1 } mxq_rule; /* ignored for NVFP4 */
+typedef enum { MXQ_OUT_BF16 = 0, MXQ_OUT_FP32 = 1 } mxq_out;
+typedef enum { MXQ_SF_ROWMAJOR = 0, MXQ_SF_SWIZZLED = 1 } mxq_sf_layout;
+
+#define MXQ_OK 0
+#define MXQ_ERR_NULL (-1)        /* a required pointer is NULL */
+#define MXQ_ERR_SHAPE (-2)       /* M, N or K out of range, or K not a multiple of what fmt needs */
+#define MXQ_ERR_ALIGN (-3)       /* a pointer is not 16-byte aligned */
+#define MXQ_ERR_UNSUPPORTED (-4) /* unknown fmt / rule / out / layout */
+#define MXQ_ERR_WORKSPACE (-5)   /* workspace smaller than mxq_linear_workspace_size() */
+#define MXQ_ERR_CUDA (-6)        /* a CUDA launch or query failed */
+#define MXQ_ERR_TIMEOUT (-7)     /* a kernel gave up on a bounded wait (see mxq_device_status) */
+#define MXQ_ERR_DEVICE (-8)      /* the current device is not sm_100 */
+
+/* Block size along K: 32 for MXFP4/MXFP8, 16 for NVFP4. */
+int mxq_block_size(mxq_fmt fmt);
+
+/* Bytes of quantized element data for a [rows, K] matrix (rows*K/2 for FP4, rows*K for MXFP8). */
+int mxq_q_bytes(int64_t rows, int64_t K, mxq_fmt fmt, size_t* bytes);
+
+/* Bytes of the scale tensor for a [rows, K] matrix in the given layout (swizzled is padded). */
+int mxq_sf_bytes(int64_t rows, int64_t K, mxq_fmt fmt, mxq_sf_layout layout, size_t* bytes);
+
+/*
+ * Quantize x [M, K] bf16 (device, row-major, K contiguous) along K.
+ *   fmt, rule     element format and MX scale rule (rule ignored for NVFP4).
+ *   global_scale  (device) fp32[1], the NVFP4 decode-direction global scale g > 0; NULL otherwise.
+ *   q_out         (device) mxq_q_bytes() bytes; sf_out (device) mxq_sf_bytes(layout) bytes.
+ * Requires M >= 1 and K >= bs with K % bs == 0.  The activation path ("Qwen3.5-9B-MXFP4-QAD-W4A4-
+ * LR1e-5-s3000", "Training mode") is fmt=MXFP4, rule=CEIL; the RTN weight export
+ * ("Qwen3.5-27B-NVFP4-RTN-weight-only", Training row: round-to-nearest) is rule=EVEN.
+ */
+int mxq_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule rule,
+                 const float* global_scale, void* q_out, void* sf_out, mxq_sf_layout layout,
+                 mxq_stream_t stream);
+
+/* Re-lay row-major scales [rows, kblocks] (device) into the swizzled tensor-core layout
+ * (device, mxq_sf_bytes(SWIZZLED) bytes, padding zeroed).  Pure byte permutation. */
+int mxq_swizzle_scales(const uint8_t* sf_rowmajor, int64_t rows, int64_t kblocks, uint8_t* sf_swizzled,
+                       mxq_stream_t stream);
+
+/*
+ * NVFP4 per-tensor global scale of x (n bf16 values, device): amax_out = max |x| and
+ * g_out = fl(amax / (6 * 448)) in fp32 (decode direction), both device fp32[1].  This is the
+ * running-max form of input_global_scale ("Qwen3.5-27B-NVFP4-GPTQ", Serving-KL table, RTN row).
+ */
+int mxq_global_scale(const void* x_bf16, int64_t n, float* g_out, float* amax_out, mxq_stream_t stream);
+
+/*
+ * Block-scaled GEMM on the tcgen05 tensor cores: out[M, N] = alpha * dq(A) dq(B)^T, fp32
+ * accumulation, alpha = g_A[0] * g_B[0] for NVFP4 and 1 otherwise ("Qwen3.5-9B-MXFP4-QAD-W4A4-
+ * LR1e-5-s3000", Serving: FP4 GEMM on quantized activations and weights).
+ *   A_q [M, K] and B_q [N, K] quantized data (device); A_sf, B_sf SWIZZLED scales (device).
+ *   g_A, g_B  (device) fp32[1] NVFP4 global scales; ignored (may be NULL) for MX formats.
+ *   out       (device) [M, N] bf16 (RNE) or fp32, row-major.
+ * Requires M, N >= 1; K >= 64 with K % 64 == 0 for FP4 and K % 32 == 0 for MXFP8.  There is no
+ * lower bound on N beyond 1.
+ */
+int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_t* B_sf, const float* g_A,
+             const float* g_B, int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_out out_type, void* out,
+             mxq_stream_t stream);
+
+/* Workspace bytes mxq_linear needs for M tokens of width K (quantized A plus swizzled scales). */
+size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt);
+
+/*
+ * Quantized linear layer: quantize x [M, K] bf16 per token with act_rule (MX) or global scale g_A
+ * (NVFP4, device fp32[1]) into `workspace`, then out = A_q * W_q^T through mxq_gemm.
+ * W_q / W_sf are the pre-quantized weights (SWIZZLED scales), g_W their NVFP4 global scale.
+ * The activation quantizer and the GEMM run back to back on `stream` with programmatic
+ * dependent launch; A is quantized once, not once per output tile.
+ */
+int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
+               int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule, mxq_out out_type,
+               void* workspace, size_t ws_bytes, void* out, mxq_stream_t stream);
+
+/* Read the device status word that kernels set when a bounded wait gives up (0 = clean).
+ * Synchronizes `stream`.  If reset != 0 the word is cleared afterwards. */
+int mxq_device_status(int* status_out, int reset, mxq_stream_t stream);
+
+/* Self-test of the bounded-wait path: launches one CTA that waits on a barrier nothing completes,
+ * with a limit of timeout_ns; the kernel records MXQ_ERR_TIMEOUT in the status word and returns.
+ * Returns MXQ_OK if the launch succeeded (read the outcome with mxq_device_status). */
+int mxq_selftest_timeout(uint64_t timeout_ns, mxq_stream_t stream);
+
+/* Human-readable name of an MXQ_* code. */
+const char* mxq_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXQ_H */

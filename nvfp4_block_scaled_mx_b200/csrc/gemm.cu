@@ -1,0 +1,430 @@
+// gemm.cu -- block-scaled GEMM on the sm_100a tensor cores (tcgen05), out = alpha * dq(A) dq(B)^T.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: A and B tiles (128-byte K slices, 128B-swizzled) and their
+//               swizzled scale tiles (bulk copies) into a STAGES-deep shared-memory ring;
+//   warp 1      TMEM owner and MMA issuer: copies each stage's scales into TMEM
+//               (tcgen05.cp 32x128b.warpx4) and issues 4 block-scaled MMAs per stage into an
+//               fp32 accumulator of 128 lanes x BN columns;
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (two warps per 32-lane sub-partition, each
+//               owning half of the BN columns), alpha scaling, bf16 RNE or fp32 conversion,
+//               stores with M/N tail masking.
+// Tiles are 128 x BN (BN = 256 or 128) and walked M-fastest so the CTAs resident at one time
+// share the same few B tiles and all of A through L2.
+//
+// Formats (KIND): 0 MXFP4 kind::mxf4 (E2M1 x E2M1, UE8M0 per 32, K = 64 per MMA)
+//                 1 NVFP4 kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 per 16, K = 64 per MMA)
+//                 2 MXFP8 kind::mxf8f6f4 (E4M3 x E4M3, UE8M0 per 32, K = 32 per MMA)
+// Every stage holds 128 bytes of K per row (256 FP4 or 128 FP8 elements), i.e. 4 MMAs.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+
+namespace mxq {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (2 + kEpiWarps) * 32;
+
+template <int KIND>
+struct Fmt;
+template <>
+struct Fmt<0> {
+    static constexpr int BS = 32, EPB = 2, MMA_K = 64;
+};
+template <>
+struct Fmt<1> {
+    static constexpr int BS = 16, EPB = 2, MMA_K = 64;
+};
+template <>
+struct Fmt<2> {
+    static constexpr int BS = 32, EPB = 1, MMA_K = 32;
+};
+
+template <int KIND, int BN, int STAGES>
+struct Cfg {
+    static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
+    static constexpr int BK = 128 * EPB;          // elements of K per stage
+    static constexpr int KSTEPS = BK / MMA_K;     // MMAs per stage (4)
+    static constexpr int KB_PER_MMA = MMA_K / BS; // scale blocks per MMA and row (2 / 4 / 1)
+    static constexpr int SF_ATOMS = BK / BS / 4;  // 512-byte scale tiles per 128 rows per stage
+    static constexpr int BGROUPS = BN / 128;
+    static constexpr int A_BYTES = kBM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SFA_BYTES = SF_ATOMS * 512;
+    static constexpr int SFB_BYTES = SF_ATOMS * BGROUPS * 512;
+    static constexpr int ACC_STAGES = (BN == 256) ? 1 : 2;
+    // TMEM columns: accumulators first, then one scale slot per pipeline stage.
+    static constexpr int SF_COLS_A = SF_ATOMS * 4;
+    static constexpr int SF_COLS_B = SF_ATOMS * (BN / 32);
+    static constexpr int SF_COLS_STAGE = SF_COLS_A + SF_COLS_B;
+    static constexpr int SF_TMEM_BASE = ACC_STAGES * BN;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(SF_TMEM_BASE + STAGES * SF_COLS_STAGE <= 512, "TMEM budget");
+    static_assert(KSTEPS == 4, "4 MMAs per 128-byte stage");
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int N_BARS = 2 * STAGES + 2 * ACC_STAGES;
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;  // + slack for 1024-byte alignment
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct GemmArgs {
+    const uint8_t* a_sf;
+    const uint8_t* b_sf;
+    const float* g_a;
+    const float* g_b;
+    void* out;
+    int M, N, K;
+    int sf_col_tiles;  // ceil(K / bs / 4)
+    int b_row_tiles;   // ceil(N / 128)
+    int m_tiles, n_tiles, k_stages;
+    int* status;
+};
+
+template <int KIND, int BN, int STAGES, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                const GemmArgs p) {
+    using C = Cfg<KIND, BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* accf = empty + STAGES;
+    uint64_t* acce = accf + C::ACC_STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_a);
+        prefetch_tmap(&tma_b);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < C::ACC_STAGES; ++a) {
+            mbar_init(&accf[a], 1);
+            mbar_init(&acce[a], kEpiWarps * 32);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // operands may come from the kernel launched just before this one on the stream
+    pdl_wait();
+
+    const int num_tiles = p.m_tiles * p.n_tiles;
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();
+            const uint64_t pol_b = policy_evict_normal();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+                int groups = 0;
+#pragma unroll
+                for (int g = 0; g < C::BGROUPS; ++g) groups += (nt * C::BGROUPS + g < p.b_row_tiles) ? 1 : 0;
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
+                    const uint32_t bytes = C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + groups);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES, ks * 128, mt * kBM, pol_a);
+                    tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, nt * BN, pol_b);
+                    const int64_t kcol = static_cast<int64_t>(ks) * C::SF_ATOMS;
+                    bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES,
+                              p.a_sf + (static_cast<int64_t>(mt) * p.sf_col_tiles + kcol) * 512, atoms * 512,
+                              &full[stage]);
+                    for (int g = 0; g < groups; ++g)
+                        bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
+                                  p.b_sf + (static_cast<int64_t>(nt * C::BGROUPS + g) * p.sf_col_tiles + kcol) * 512,
+                                  atoms * 512, &full[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int nt = tile / p.m_tiles;
+                int groups = 0;
+#pragma unroll
+                for (int g = 0; g < C::BGROUPS; ++g) groups += (nt * C::BGROUPS + g < p.b_row_tiles) ? 1 : 0;
+                if (!mbar_wait(&acce[acc], acc_phase ^ 1u, p.status, 2)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, p.status, 3)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
+                    const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+                    const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+                    for (int a = 0; a < atoms; ++a)
+                        tc_cp_scales(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
+                    for (int g = 0; g < groups; ++g)
+                        for (int a = 0; a < atoms; ++a)
+                            tc_cp_scales(sf_col + C::SF_COLS_A + a * (BN / 32) + g * 4,
+                                         smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                    const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                    const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+#pragma unroll
+                    for (int j = 0; j < C::KSTEPS; ++j) {
+                        if (ks * C::BK + j * C::MMA_K < p.K) {
+                            const int kb = j * C::KB_PER_MMA;  // first scale block of this MMA in the stage
+                            const int atom = kb >> 2;
+                            const uint32_t idesc = mma_idesc<KIND>(kBM, BN, static_cast<uint32_t>(kb & 3));
+                            mma_block_scaled<KIND>(d_tmem, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                                   smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B), idesc,
+                                                   sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * (BN / 32),
+                                                   (ks | j) != 0 ? 1u : 0u);
+                        }
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&accf[acc]);
+                if (++acc == C::ACC_STAGES) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        constexpr int COLS = BN / 2;  // accumulator columns owned by this warp
+        const int sub = warp & 3;     // TMEM sub-partition this warp may read
+        const int col0 = ((warp - 2) >> 2) * COLS;
+        const int row = sub * 32 + lane;
+        const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+            if (!mbar_wait(&accf[acc], acc_phase, p.status, 4)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
+                                   static_cast<uint32_t>(acc * BN + col0);
+            const int m = mt * kBM + row;
+            const int n0 = nt * BN + col0;
+            if constexpr (!OUT_F32) {
+                uint32_t packed[COLS / 2];
+#pragma unroll
+                for (int c = 0; c < COLS / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
+                        if (KIND == 1) {
+                            lo = __fmul_rn(lo, alpha);
+                            hi = __fmul_rn(hi, alpha);
+                        }
+                        const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                        packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
+                    }
+                }
+                // the accumulator is free for the next tile once it sits in registers
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+                if (m < p.M) {
+                    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
+                    if (n0 + COLS <= p.N && (p.N & 7) == 0) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + n0);
+#pragma unroll
+                        for (int v = 0; v < COLS / 8; ++v)
+                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+                        uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+#pragma unroll
+                        for (int v = 0; v < COLS / 2; ++v) {
+                            const int n = n0 + 2 * v;
+                            if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                            if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                        }
+                    }
+                }
+            } else {
+                float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(m) * p.N;
+                const bool vec = (p.N & 3) == 0;
+#pragma unroll 1
+                for (int c = 0; c < COLS / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        const int nb = n0 + c * 32;
+                        if (vec && nb + 32 <= p.N) {
+                            float4* dst = reinterpret_cast<float4*>(orow + nb);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                float4 f;
+                                f.x = __fmul_rn(__uint_as_float(r[4 * v]), alpha);
+                                f.y = __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha);
+                                f.z = __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha);
+                                f.w = __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha);
+                                dst[v] = f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (nb + i < p.N) orow[nb + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+            }
+            if (++acc == C::ACC_STAGES) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes], box of 128 bytes x box_rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND, int BN, int STAGES, bool F32>
+int run(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t stream, bool pdl) {
+    using C = Cfg<KIND, BN, STAGES>;
+    auto kern = gemm_kernel<KIND, BN, STAGES, F32>;
+    const int row_bytes = args.K / C::EPB;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A_q, row_bytes, args.M, kBM) || !make_map(&tb, B_q, row_bytes, args.N, BN)) return MXQ_ERR_CUDA;
+    args.m_tiles = static_cast<int>(ceil_div(args.M, kBM));
+    args.n_tiles = static_cast<int>(ceil_div(args.N, BN));
+    args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = static_cast<int64_t>(args.m_tiles) * args.n_tiles;
+    const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
+template <int KIND, bool F32>
+int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
+    // 256-wide tiles when they still give at least two waves of work, 128-wide otherwise
+    const int64_t tiles256 = ceil_div(args.M, kBM) * ceil_div(args.N, 256);
+    if (tiles256 >= 2 * static_cast<int64_t>(sm_count())) return run<KIND, 256, 4, F32>(A_q, B_q, args, stream, pdl);
+    return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);
+}
+
+}  // namespace
+
+int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_t* B_sf, const float* g_A,
+                const float* g_B, int64_t M, int64_t N, int64_t K, int fmt, int out_type, void* out,
+                cudaStream_t stream, bool pdl_secondary) {
+    GemmArgs a = {};
+    a.a_sf = A_sf;
+    a.b_sf = B_sf;
+    a.g_a = g_A;
+    a.g_b = g_B;
+    a.out = out;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.sf_col_tiles = static_cast<int>(ceil_div(K / block_size(fmt), 4));
+    a.b_row_tiles = static_cast<int>(ceil_div(N, 128));
+    a.status = status_ptr();
+    const bool f32 = out_type == MXQ_OUT_FP32;
+    switch (fmt) {
+        case MXQ_MXFP4:
+            return f32 ? dispatch_bn<0, true>(A_q, B_q, a, stream, pdl_secondary)
+                       : dispatch_bn<0, false>(A_q, B_q, a, stream, pdl_secondary);
+        case MXQ_NVFP4:
+            return f32 ? dispatch_bn<1, true>(A_q, B_q, a, stream, pdl_secondary)
+                       : dispatch_bn<1, false>(A_q, B_q, a, stream, pdl_secondary);
+        default:
+            return f32 ? dispatch_bn<2, true>(A_q, B_q, a, stream, pdl_secondary)
+                       : dispatch_bn<2, false>(A_q, B_q, a, stream, pdl_secondary);
+    }
+}
+
+}  // namespace mxq

@@ -1,0 +1,42 @@
+// mxq_internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mxq.h"
+
+namespace mxq {
+
+// Device status word of the current device (kernels record bounded-wait timeouts there).
+int* status_ptr();
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline int block_size(int fmt) { return fmt == MXQ_NVFP4 ? 16 : 32; }
+
+inline int64_t swizzled_sf_bytes(int64_t rows, int64_t kblocks) {
+    return ceil_div(rows, 128) * 128 * ceil_div(kblocks, 4) * 4;
+}
+
+// Quantizer launch (arguments already validated).  `pdl_primary` lets a dependent kernel launched
+// with programmatic stream serialization start early.
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q,
+                            void* sf, int layout, cudaStream_t stream);
+
+cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream);
+
+cudaError_t launch_global_scale(const void* x, int64_t n, float* g_out, float* amax_out, cudaStream_t stream);
+
+// GEMM launch.  `pdl_secondary` launches with programmatic stream serialization so that the
+// kernel's prologue overlaps the tail of the preceding kernel on the stream.
+int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_t* B_sf, const float* g_A,
+                const float* g_B, int64_t M, int64_t N, int64_t K, int fmt, int out_type, void* out,
+                cudaStream_t stream, bool pdl_secondary);
+
+cudaError_t launch_selftest_timeout(uint64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace mxq

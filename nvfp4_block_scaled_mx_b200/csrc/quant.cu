@@ -1,0 +1,254 @@
+// quant.cu -- bf16 -> MXFP4 (EVEN / CEIL), NVFP4 and MXFP8 block quantizer, scale swizzle,
+// NVFP4 global scale, and the bounded-wait self-test kernel.
+//
+// The quantizer is a single streaming pass over x: each thread owns 8 consecutive elements
+// (one 16-byte load); the bs/8 threads of a block reduce the block amax on the bf16 bit patterns
+// with warp shuffles, derive the scale, and write packed codes (4 bytes per thread for FP4,
+// 8 for FP8) plus one scale byte per block, either row-major or directly in the swizzled
+// tensor-core layout.  Loads of one warp cover 512 contiguous bytes; stores 128 (FP4) or 256 bytes.
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+
+namespace mxq {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Scale byte offset of block (row, kc) in the swizzled layout.
+__device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t kc, uint32_t col_tiles) {
+    return ((row >> 7) * col_tiles + (kc >> 2)) * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + (kc & 3u);
+}
+
+template <int FMT, int RULE, bool SWZ>
+__device__ __forceinline__ void quantize_chunk(const uint4 v, const int64_t ci, const bool ok, const uint32_t kblocks,
+                                               const uint32_t col_tiles, const float g, uint8_t* __restrict__ q,
+                                               uint8_t* __restrict__ sf) {
+    constexpr int BS = (FMT == MXQ_NVFP4) ? 16 : 32;
+    constexpr int LPB = BS / 8;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // block amax on |bf16| bit patterns (non-negative floats order like their bits)
+    const uint32_t m2 = __vmaxu2(__vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
+                                 __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
+    uint32_t amax16 = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+    for (int off = 1; off < LPB; off <<= 1) amax16 = max(amax16, __shfl_xor_sync(0xFFFFFFFFu, amax16, off));
+    const uint32_t abits = amax16 << 16;
+
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+
+    uint32_t scale_byte;
+    if constexpr (FMT == MXQ_NVFP4) {
+        const float amax = __uint_as_float(abits);
+        uint32_t s = 0;
+        if (amax != 0.0f) {
+            const float t = __fdiv_rn(amax, 6.0f);
+            const float u = __fdiv_rn(t, g);
+            s = cvt_e4m3x2(u, 0.0f) & 0xFFu;
+        }
+        const float d = __fmul_rn(e4m3_decode_pos(s), g);
+        uint32_t packed;
+        if (d == 0.0f) {
+            packed = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) packed |= (__float_as_uint(f[i]) >> 31) << (4 * i + 3);
+        } else {
+            const float r = __fdiv_rn(1.0f, d);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], r);
+            packed = cvt_e2m1x8(f);
+        }
+        scale_byte = s;
+        if (ok) reinterpret_cast<uint32_t*>(q)[ci] = packed;
+    } else {
+        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
+        // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
+        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
+        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
+        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
+        e = max(e, -127);
+        const float inv = exp2_neg(e);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], inv);
+        scale_byte = static_cast<uint32_t>(e + 127);
+        if constexpr (FMT == MXQ_MXFP8) {
+            const uint32_t lo = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
+            const uint32_t hi = cvt_e4m3x2(f[4], f[5]) | (cvt_e4m3x2(f[6], f[7]) << 16);
+            if (ok) reinterpret_cast<uint2*>(q)[ci] = make_uint2(lo, hi);
+        } else {
+            if (ok) reinterpret_cast<uint32_t*>(q)[ci] = cvt_e2m1x8(f);
+        }
+    }
+    if (ok && (threadIdx.x % LPB) == 0) {
+        const uint32_t blk = static_cast<uint32_t>(ci / LPB);
+        uint32_t off = blk;
+        if constexpr (SWZ) {
+            const uint32_t row = blk / kblocks;
+            const uint32_t kc = blk - row * kblocks;
+            off = swz_offset(row, kc, col_tiles);
+        }
+        sf[off] = static_cast<uint8_t>(scale_byte);
+    }
+}
+
+template <int FMT, int RULE, bool SWZ>
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __restrict__ x, int64_t n_chunks,
+                                                                 uint32_t kblocks, uint32_t col_tiles,
+                                                                 const float* __restrict__ gptr,
+                                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    pdl_launch_dependents();
+    const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    // warp-uniform loop bound so that every lane takes part in the shuffles
+    for (int64_t wbase = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); wbase < n_chunks;
+         wbase += kQuantUnroll * stride) {
+        uint4 v[kQuantUnroll];
+        bool ok[kQuantUnroll];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t ci = wbase + lane + u * stride;
+            ok[u] = ci < n_chunks;
+            v[u] = ok[u] ? ld_stream(x + ci) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u)
+            quantize_chunk<FMT, RULE, SWZ>(v[u], wbase + lane + u * stride, ok[u], kblocks, col_tiles, g, q, sf);
+    }
+}
+
+template <int FMT, int RULE, bool SWZ>
+cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, cudaStream_t stream) {
+    const int64_t n_chunks = M * K / 8;
+    const uint32_t kblocks = static_cast<uint32_t>(K / block_size(FMT));
+    const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
+    int64_t blocks = ceil_div(n_chunks, static_cast<int64_t>(kQuantThreads) * kQuantUnroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    quantize_kernel<FMT, RULE, SWZ><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), n_chunks, kblocks, col_tiles, g, static_cast<uint8_t*>(q),
+        static_cast<uint8_t*>(sf));
+    return cudaGetLastError();
+}
+
+template <bool SWZ>
+cudaError_t launch_q_layout(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q, void* sf,
+                            cudaStream_t stream) {
+    if (fmt == MXQ_NVFP4) return launch_q<MXQ_NVFP4, 0, SWZ>(x, M, K, g, q, sf, stream);
+    if (fmt == MXQ_MXFP8) {
+        return rule == MXQ_RULE_CEIL ? launch_q<MXQ_MXFP8, MXQ_RULE_CEIL, SWZ>(x, M, K, g, q, sf, stream)
+                                     : launch_q<MXQ_MXFP8, MXQ_RULE_EVEN, SWZ>(x, M, K, g, q, sf, stream);
+    }
+    return rule == MXQ_RULE_CEIL ? launch_q<MXQ_MXFP4, MXQ_RULE_CEIL, SWZ>(x, M, K, g, q, sf, stream)
+                                 : launch_q<MXQ_MXFP4, MXQ_RULE_EVEN, SWZ>(x, M, K, g, q, sf, stream);
+}
+
+// ------------------------------------------------------------------ swizzle
+
+__global__ void swizzle_kernel(const uint8_t* __restrict__ src, uint32_t rows, uint32_t kblocks, uint32_t col_tiles,
+                               uint8_t* __restrict__ dst, int64_t total) {
+    for (int64_t off = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; off < total;
+         off += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t tile = static_cast<uint32_t>(off >> 9), within = static_cast<uint32_t>(off & 511);
+        const uint32_t rt = tile / col_tiles, ct = tile - rt * col_tiles;
+        const uint32_t r = rt * 128u + ((within & 15u) >> 2) * 32u + (within >> 4);
+        const uint32_t c = ct * 4u + (within & 3u);
+        dst[off] = (r < rows && c < kblocks) ? src[static_cast<int64_t>(r) * kblocks + c] : 0;
+    }
+}
+
+// ------------------------------------------------------------------ global scale
+
+__global__ void amax_kernel(const uint4* __restrict__ x, int64_t n_chunks, const uint16_t* __restrict__ tail,
+                            int n_tail, unsigned int* __restrict__ amax_bits) {
+    uint32_t m = 0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 v = ld_stream(x + i);
+        const uint32_t m2 = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                     __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+        m = max(m, max(m2 & 0xFFFFu, m2 >> 16));
+    }
+    if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < n_tail) m = max(m, static_cast<uint32_t>(tail[threadIdx.x] & 0x7FFFu));
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_bits, m << 16);
+}
+
+__global__ void global_scale_finalize(const float* amax, float* g) { *g = __fdiv_rn(*amax, 2688.0f); }
+
+// ------------------------------------------------------------------ bounded-wait self-test
+
+__global__ void selftest_timeout_kernel(int* status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // phase 0 of this barrier never completes: nothing arrives on it
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, status, 99, limit_ns);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q, void* sf,
+                            int layout, cudaStream_t stream) {
+    if (layout == MXQ_SF_SWIZZLED) {
+        const int64_t kb = K / block_size(fmt);
+        if (M % 128 != 0 || kb % 4 != 0) {
+            cudaError_t e = cudaMemsetAsync(sf, 0, static_cast<size_t>(swizzled_sf_bytes(M, kb)), stream);
+            if (e != cudaSuccess) return e;
+        }
+        return launch_q_layout<true>(x, M, K, fmt, rule, g, q, sf, stream);
+    }
+    return launch_q_layout<false>(x, M, K, fmt, rule, g, q, sf, stream);
+}
+
+cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream) {
+    const int64_t total = swizzled_sf_bytes(rows, kblocks);
+    int64_t blocks = ceil_div(total, 256);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    if (blocks > cap) blocks = cap;
+    swizzle_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        src, static_cast<uint32_t>(rows), static_cast<uint32_t>(kblocks), static_cast<uint32_t>(ceil_div(kblocks, 4)),
+        dst, total);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_global_scale(const void* x, int64_t n, float* g_out, float* amax_out, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    const int64_t n_chunks = n / 8;
+    const int n_tail = static_cast<int>(n - n_chunks * 8);
+    int64_t blocks = ceil_div(n_chunks > 0 ? n_chunks : 1, 256 * 4);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint4*>(x), n_chunks, static_cast<const uint16_t*>(x) + n_chunks * 8, n_tail,
+        reinterpret_cast<unsigned int*>(amax_out));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    global_scale_finalize<<<1, 1, 0, stream>>>(amax_out, g_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_timeout(uint64_t timeout_ns, cudaStream_t stream) {
+    selftest_timeout_kernel<<<1, 32, 0, stream>>>(status_ptr(), timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace mxq

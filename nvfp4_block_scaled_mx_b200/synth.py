@@ -36,7 +36,7 @@ CONFIGS = {
 _CHUNK_ROWS = 4096
 
 
-def _draw(kind, rows, K, gen, device, std=1.0, **_):
+def _draw(rows, K, gen, device, kind, std=1.0, **_):
     if kind == "normal":
         return torch.randn(rows, K, generator=gen, device=device) * std
     if kind == "student_t3":
@@ -54,7 +54,7 @@ def draw_matrix(rows, K, spec, gen, device="cpu"):
     out = torch.empty(rows, K, dtype=torch.bfloat16, device=device)
     for r0 in range(0, rows, _CHUNK_ROWS):
         r1 = min(rows, r0 + _CHUNK_ROWS)
-        out[r0:r1] = _draw(spec["kind"], r1 - r0, K, gen, device, **spec).to(torch.bfloat16)
+        out[r0:r1] = _draw(r1 - r0, K, gen, device, **spec).to(torch.bfloat16)
     frac = spec.get("outlier_frac", 0.0)
     if frac > 0:
         n_out = int(round(frac * K))

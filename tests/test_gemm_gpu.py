@@ -1,0 +1,194 @@
+"""GPU parity of the tcgen05 block-scaled GEMM (mxq_gemm) and the fused linear (mxq_linear)
+against the oracle's fp64 GEMM of the dequantized operands.
+
+Tolerance: fp32 output |gpu - ref| <= 2^-20 * sum_k |a_k b_k|; bf16 output within one bf16 ulp of
+ref on top of that fp32 allowance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_scaled_mx_b200 import mxq, synth
+from tests.helpers import FMTS, RULES, check_bf16, check_fp32, oracle_quantize, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _quant_pair(A, W, fmt, a_rule, w_rule):
+    gA = gW = 1.0
+    if fmt == "nvfp4":
+        gA, _ = oracle.global_scale(A)
+        gW, _ = oracle.global_scale(W)
+    Aq, Asf = oracle_quantize(A, fmt, a_rule, gA)
+    Wq, Wsf = oracle_quantize(W, fmt, w_rule, gW)
+    return (Aq, Asf, float(gA)), (Wq, Wsf, float(gW))
+
+
+def _gpu_gemm(a, w, M, N, K, fmt, out_dtype):
+    (Aq, Asf, gA), (Wq, Wsf, gW) = a, w
+    dev = lambda z: torch.from_numpy(np.ascontiguousarray(z)).cuda()
+    g_a = torch.tensor([gA], dtype=torch.float32, device="cuda")
+    g_w = torch.tensor([gW], dtype=torch.float32, device="cuda")
+    out = mxq.gemm(dev(Aq), dev(oracle.swizzle(Asf)), dev(Wq), dev(oracle.swizzle(Wsf)), M, N, K, fmt,
+                   out_dtype=out_dtype, g_A=g_a, g_B=g_w)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy() if out_dtype == torch.bfloat16 else to_np(out).astype(np.float64)
+
+
+SHAPES = [(1, 1, 64), (16, 256, 256), (128, 128, 128), (200, 300, 320), (129, 520, 1024), (300, 257, 576),
+          (64, 96, 5120), (512, 768, 192)]
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_gemm_matches_oracle(fmt, out_dtype, shape):
+    M, N, K = shape
+    if fmt == "mxfp8" and K % 32:
+        pytest.skip()
+    A = synth.random_bf16((M, K), M + 3 * N + K, std=1.0)
+    W = synth.random_bf16((N, K), M + 5 * N + K, std=0.02)
+    a, w = _quant_pair(A, W, fmt, "ceil", "even")
+    ref, abs_sum = oracle.gemm(a[0], a[1], w[0], w[1], M, N, K, FMTS[fmt], gA=a[2], gB=w[2])
+    gpu = _gpu_gemm(a, w, M, N, K, fmt, out_dtype)
+    if out_dtype == torch.float32:
+        check_fp32(gpu, ref, abs_sum, "%s %s" % (fmt, shape))
+    else:
+        check_bf16(gpu, ref, abs_sum, "%s %s" % (fmt, shape))
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+def test_gemm_unit_scales_exact(fmt):
+    """Unit scales and small integer-valued codes: every partial sum is exact in fp32, so the
+    GPU result must equal the oracle exactly (pins operand layout and nibble order)."""
+    M, N, K = 130, 260, 512
+    rng = np.random.default_rng(7)
+    bs = 16 if fmt == "nvfp4" else 32
+    if fmt == "mxfp8":
+        Aq = rng.integers(0, 256, (M, K), dtype=np.uint8)
+        Wq = rng.integers(0, 256, (N, K), dtype=np.uint8)
+        # normal E4M3 codes with exponent field 8 only: |v| in [2, 3.75], multiples of 1/4
+        Aq = (Aq & 0x87) | 0x40
+        Wq = (Wq & 0x87) | 0x40
+        one = 127
+    else:
+        Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+        Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+        one = 127 if fmt == "mxfp4" else 0x38  # E8M0 1.0 or E4M3 1.0
+    Asf = np.full((M, K // bs), one, np.uint8)
+    Wsf = np.full((N, K // bs), one, np.uint8)
+    ref, abs_sum = oracle.gemm(Aq, Asf, Wq, Wsf, M, N, K, FMTS[fmt])
+    gpu = _gpu_gemm((Aq, Asf, 1.0), (Wq, Wsf, 1.0), M, N, K, fmt, torch.float32)
+    assert np.array_equal(gpu, ref), "max abs diff %g" % np.abs(gpu - ref).max()
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+def test_gemm_scale_placement(fmt):
+    """Distinct power-of-two scales per (row, block) on one operand at a time: pins how the
+    swizzled scale tiles map to rows and K blocks inside the MMA."""
+    M, N, K = 256, 256, 1024
+    bs = 16 if fmt == "nvfp4" else 32
+    rng = np.random.default_rng(3)
+    A = synth.random_bf16((M, K), 21)
+    W = synth.random_bf16((N, K), 22, std=0.02)
+    a, w = _quant_pair(A, W, fmt, "even", "even")
+    for side in ("A", "B"):
+        Aq, Asf, gA = a
+        Wq, Wsf, gW = w
+        if fmt == "nvfp4":
+            codes = np.array([0x30, 0x38, 0x40, 0x48, 0x28], np.uint8)  # 0.5, 1, 2, 4, 0.25
+        else:
+            codes = np.array([125, 126, 127, 128, 129, 130], np.uint8)
+        if side == "A":
+            Asf = rng.choice(codes, Asf.shape).astype(np.uint8)
+        else:
+            Wsf = rng.choice(codes, Wsf.shape).astype(np.uint8)
+        ref, abs_sum = oracle.gemm(Aq, Asf, Wq, Wsf, M, N, K, FMTS[fmt], gA=gA, gB=gW)
+        gpu = _gpu_gemm((Aq, Asf, gA), (Wq, Wsf, gW), M, N, K, fmt, torch.float32)
+        check_fp32(gpu, ref, abs_sum, "%s scales on %s" % (fmt, side))
+
+
+@pytest.mark.parametrize("fmt,M,N,K", [("mxfp4", 16, 256, 256), ("mxfp4", 200, 333, 640), ("nvfp4", 130, 520, 1024),
+                                       ("mxfp8", 64, 96, 512)])
+def test_linear_matches_oracle(fmt, M, N, K):
+    """mxq_linear (dynamic activation quantization + GEMM) == oracle quantize + fp64 GEMM."""
+    A = synth.random_bf16((M, K), 99 + M, std=1.0)
+    W = synth.random_bf16((N, K), 98 + N, std=0.02)
+    a, w = _quant_pair(A, W, fmt, "ceil", "even")
+    ref, abs_sum = oracle.gemm(a[0], a[1], w[0], w[1], M, N, K, FMTS[fmt], gA=a[2], gB=w[2])
+    Wd = W.cuda()
+    g_w = g_a = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(Wd)
+        g_a, _ = mxq.global_scale(A.cuda())
+    Wq, Wsf = mxq.quantize(Wd, fmt, "even", global_scale=g_w, layout=mxq.SF_SWIZZLED)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out = mxq.linear(A.cuda(), Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+        torch.cuda.synchronize()
+        gpu = out.double().cpu().numpy()
+        if out_dtype == torch.float32:
+            check_fp32(gpu, ref, abs_sum, "linear %s" % fmt)
+        else:
+            check_bf16(gpu, ref, abs_sum, "linear %s" % fmt)
+
+
+def test_tiny_config_full():
+    """The tiny MXFP4 W4A4 linear problem: every output element, fp32 out."""
+    cfg = synth.CONFIGS["tiny"]
+    A, W = synth.make_inputs("tiny")
+    M, N, K = cfg["M"], cfg["N"], cfg["K"]
+    a, w = _quant_pair(A, W, "mxfp4", "ceil", "even")
+    ref, abs_sum = oracle.gemm(a[0], a[1], w[0], w[1], M, N, K, oracle.MXFP4)
+    Wq, Wsf = mxq.quantize(W.cuda(), "mxfp4", "even")
+    out = mxq.linear(A.cuda(), Wq, Wsf, N, "mxfp4", act_rule="ceil", out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    check_fp32(to_np(out).astype(np.float64), ref, abs_sum, "tiny")
+
+
+def test_bounded_wait_selftest():
+    """A kernel waiting on a barrier nothing completes gives up after its limit and reports
+    MXQ_ERR_TIMEOUT through the status word; the context stays usable."""
+    mxq.mxq_device_status(reset=True)
+    mxq.mxq_selftest_timeout(20_000_000)  # 20 ms
+    st = mxq.mxq_device_status(reset=True)
+    assert st == 0x100 + 99
+    assert mxq.mxq_device_status(reset=False) == 0
+    x = torch.ones(4, 64, dtype=torch.bfloat16, device="cuda")
+    q, sf = mxq.quantize(x, "mxfp4", "ceil", layout=mxq.SF_ROWMAJOR)
+    torch.cuda.synchronize()
+    assert int(sf[0, 0]) == 125  # amax 1 -> CEIL e = -2
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill_gate_up", "down_nvfp4", "attn_mxfp8", "lm_head"])
+def test_linear_full_size_sampled(name):
+    """Each full-size problem through mxq_linear in the bench's launch configuration (weights
+    quantized on the GPU, activations quantized inside the call); a seeded sample of outputs
+    (random rows x random columns plus the last row and column) is recomputed by the oracle from
+    the bf16 inputs alone."""
+    cfg = synth.CONFIGS[name]
+    M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
+    A, W = synth.make_inputs(name, device="cuda")
+    g_w = g_a = None
+    gA = gW = 1.0
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(W)
+        g_a, _ = mxq.global_scale(A)
+        gW_ref, _ = oracle.global_scale(W.cpu())
+        gA_ref, _ = oracle.global_scale(A.cpu())
+        assert to_np(g_w)[0] == gW_ref and to_np(g_a)[0] == gA_ref
+        gA, gW = float(gA_ref), float(gW_ref)
+    Wq, Wsf = mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED)
+    out_dtype = torch.float32 if cfg["out"] == "fp32" else torch.bfloat16
+    out = mxq.linear(A, Wq, Wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+    torch.cuda.synchronize()
+    gen = torch.Generator().manual_seed(hash(name) % 1000)
+    rows = sorted(set(torch.randint(0, M, (min(M, 48),), generator=gen).tolist()) | {M - 1})
+    cols = sorted(set(torch.randint(0, N, (48,), generator=gen).tolist()) | {N - 1})
+    Aq, Asf = oracle_quantize(A[rows].cpu(), fmt, cfg["a_rule"], gA)
+    Wq_ref, Wsf_ref = oracle_quantize(W[cols].cpu(), fmt, cfg["w_rule"], gW)
+    ref, abs_sum = oracle.gemm(Aq, Asf, Wq_ref, Wsf_ref, len(rows), len(cols), K, FMTS[fmt], gA=gA, gB=gW)
+    gpu = out[rows][:, cols].double().cpu().numpy()
+    if out_dtype == torch.float32:
+        check_fp32(gpu, ref, abs_sum, name)
+    else:
+        check_bf16(gpu, ref, abs_sum, name)

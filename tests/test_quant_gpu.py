@@ -1,0 +1,115 @@
+"""GPU parity of mxq_quantize / mxq_swizzle_scales / mxq_global_scale against the CPU oracle:
+quantized bytes and scales must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_scaled_mx_b200 import mxq, synth
+from tests.helpers import FMTS, RULES, oracle_quantize, to_np
+from tests.test_oracle_quant import _adversarial_bf16
+
+pytestmark = pytest.mark.gpu
+
+COMBOS = [("mxfp4", "even"), ("mxfp4", "ceil"), ("mxfp8", "even"), ("mxfp8", "ceil"), ("nvfp4", "even")]
+
+
+def _run(x_cpu, fmt, rule, layout, g=None):
+    x = x_cpu.cuda()
+    gd = None
+    if fmt == "nvfp4":
+        gd = torch.tensor([g], dtype=torch.float32, device="cuda")
+    q, sf = mxq.quantize(x, fmt, rule, global_scale=gd, layout=layout)
+    torch.cuda.synchronize()
+    return to_np(q), to_np(sf)
+
+
+@pytest.mark.parametrize("fmt,rule", COMBOS)
+@pytest.mark.parametrize("shape", [(1, 32), (3, 64), (37, 320), (130, 1056), (256, 5120)])
+def test_quantize_matches_oracle(fmt, rule, shape):
+    M, K = shape
+    bs = 16 if fmt == "nvfp4" else 32
+    if K % bs:
+        pytest.skip("K not a multiple of the block")
+    x = _adversarial_bf16(M, K, M * 7 + K, huge=3.0e38 if fmt != "nvfp4" else 3.0e6, bs=bs)
+    g = 1.0
+    if fmt == "nvfp4":
+        g, _ = oracle.global_scale(x)
+    q_ref, sf_ref = oracle_quantize(x, fmt, rule, g)
+    for layout in (mxq.SF_ROWMAJOR, mxq.SF_SWIZZLED):
+        q, sf = _run(x, fmt, rule, layout, float(g))
+        assert np.array_equal(q, q_ref), "element codes differ (%s/%s %s)" % (fmt, rule, shape)
+        if layout == mxq.SF_ROWMAJOR:
+            assert np.array_equal(sf.reshape(sf_ref.shape), sf_ref)
+        else:
+            assert np.array_equal(sf, oracle.swizzle(sf_ref)), "swizzled scales (incl. zero padding) differ"
+
+
+@pytest.mark.parametrize("fmt,rule", COMBOS)
+def test_quantize_random_fuzz(fmt, rule):
+    """Seeded fuzz over plain Gaussian data with per-row dynamic range, many blocks."""
+    g = torch.Generator().manual_seed(11)
+    mism = 0
+    total = 0
+    for it in range(6):
+        M = int(torch.randint(1, 300, (1,), generator=g))
+        K = 64 * int(torch.randint(1, 40, (1,), generator=g))
+        x = (torch.randn(M, K, generator=g) * torch.exp(torch.randn(M, 1, generator=g) * 4)).to(torch.bfloat16)
+        gs = 1.0
+        if fmt == "nvfp4":
+            gs, _ = oracle.global_scale(x)
+        q_ref, sf_ref = oracle_quantize(x, fmt, rule, gs)
+        q, sf = _run(x, fmt, rule, mxq.SF_ROWMAJOR, float(gs))
+        mism += int((q != q_ref).sum()) + int((sf.reshape(sf_ref.shape) != sf_ref).sum())
+        total += q.size + sf.size
+    assert mism == 0, "%d / %d mismatching bytes" % (mism, total)
+
+
+def test_swizzle_kernel_matches_oracle():
+    for rows, kb in [(1, 1), (5, 3), (128, 4), (300, 160), (257, 1088)]:
+        sf = torch.randint(0, 256, (rows, kb), dtype=torch.uint8, generator=torch.Generator().manual_seed(rows))
+        out = mxq.swizzle_scales(sf.cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(to_np(out), oracle.swizzle(sf.numpy()))
+
+
+def test_global_scale_matches_oracle():
+    for n, seed in [(16, 1), (1000, 2), (8192 * 17 + 5, 3)]:
+        x = synth.random_bf16((n,), seed, std=3.0)
+        g_ref, amax_ref = oracle.global_scale(x)
+        g, amax = mxq.global_scale(x.cuda())
+        torch.cuda.synchronize()
+        assert to_np(amax)[0] == amax_ref and to_np(g)[0] == g_ref
+
+
+@pytest.mark.parametrize("name,which", [("prefill_gate_up", "A"), ("prefill_gate_up", "W"), ("down_nvfp4", "A"),
+                                        ("attn_mxfp8", "W"), ("lm_head", "W"), ("decode", "A")])
+def test_quantize_full_size_sampled_rows(name, which):
+    """Full-size tensors quantized in the bench's launch configuration; every byte of a seeded
+    sample of rows is checked against the oracle (rows quantize independently)."""
+    cfg = synth.CONFIGS[name]
+    A, W = synth.make_inputs(name, device="cuda")
+    x = A if which == "A" else W
+    del A, W
+    rule = cfg["a_rule"] if which == "A" else cfg["w_rule"]
+    fmt = cfg["fmt"]
+    gd = None
+    g = 1.0
+    if fmt == "nvfp4":
+        gd, _ = mxq.global_scale(x)
+        g = float(to_np(gd)[0])
+    q, sf = mxq.quantize(x, fmt, rule, global_scale=gd, layout=mxq.SF_SWIZZLED)
+    torch.cuda.synchronize()
+    rows_total, K = x.shape
+    gen = torch.Generator().manual_seed(123)
+    rows = torch.unique(torch.cat([torch.randint(0, rows_total, (96,), generator=gen),
+                                   torch.tensor([0, rows_total - 1])])).tolist()
+    xs = x[rows].cpu()
+    if fmt == "nvfp4":
+        g_ref, _ = oracle.global_scale(x.cpu())
+        assert np.float32(g) == g_ref
+    q_ref, sf_ref = oracle_quantize(xs, fmt, rule, g)
+    assert np.array_equal(to_np(q[rows]), q_ref)
+    kb = K // (16 if fmt == "nvfp4" else 32)
+    sf_rm = oracle.unswizzle(to_np(sf), rows_total, kb)
+    assert np.array_equal(sf_rm[rows], sf_ref)
