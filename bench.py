@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--workload", default="prefill_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--M", type=int, default=None, help="override the workload's M (profiling runs)")
+    ap.add_argument("--N", type=int, default=None, help="override the workload's N (profiling runs)")
     return ap.parse_args()
 
 
@@ -174,11 +176,14 @@ def run_mxq(args, world, rank, local):
         raise SystemExit("bench.py --impl mxq needs a CUDA device (there is no CPU fallback)")
     dev = torch.device("cuda", local)
     cfg = synth.CONFIGS[args.workload]
-    M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
+    M = args.M or cfg["M"]
+    N = args.N or cfg["N"]
+    K, fmt = cfg["K"], cfg["fmt"]
+    workload = args.workload if (M, N) == (cfg["M"], cfg["N"]) else "%s(M=%d,N=%d)" % (args.workload, M, N)
     stream = torch.cuda.current_stream(dev)
     hbm_gbs, bf16_tflops, peak_src = peaks()
 
-    A, W = synth.make_inputs(args.workload, device=dev)
+    A, W = synth.make_inputs(args.workload, device=dev, M=M, N=N)
     g_w = g_a = None
     if fmt == "nvfp4":
         g_w, _ = mxq.global_scale(W)
@@ -232,7 +237,7 @@ def run_mxq(args, world, rank, local):
                 "peak_source": "%s bf16 %.1f TFLOP/s x %g nominal %s:bf16 ratio" % (
                     peak_src, bf16_tflops, FP4_PER_BF16 if fmt != "mxfp8" else FP8_PER_BF16, fmt),
                 "frac_of_datasheet": round(gemm_tflops / (9000.0 if fmt != "mxfp8" else 4500.0), 4),
-                "traffic": traffic_for("gemm_%s_%s" % (fmt, args.workload)),
+                "traffic": traffic_for("gemm_%s_%s" % (fmt, workload)),
                 "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
@@ -255,7 +260,7 @@ def run_mxq(args, world, rank, local):
            "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "e2m1xe2m1->f32 (bf16 out)" if fmt != "mxfp8" else
            "e4m3xe4m3->f32 (bf16 out)", "data": "synthetic (seeded, random-init weights)",
-           "config": {"workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt, "act_rule": cfg["a_rule"],
+           "config": {"workload": workload, "M": M, "N": N, "K": K, "fmt": fmt, "act_rule": cfg["a_rule"],
                       "weight_rule": cfg["w_rule"], "out": cfg["out"], "l2": "working set > 126 MB L2, no flush",
                       "parallelism": "replicas x%d (no collective)" % world},
            "gpu_launches": 2 * args.steps, "roofline": roofline, "quantize": quant, "quantize_weight": quant_w,
