@@ -122,6 +122,30 @@ int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const f
                int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule, mxq_out out_type,
                void* workspace, size_t ws_bytes, void* out, mxq_stream_t stream);
 
+/*
+ * mxq_linear without a caller-supplied workspace.  The paper has no counterpart: this call exists
+ * for callers that are not allowed to allocate device memory -- e.g. plugins inside a host
+ * framework that owns all device memory and passes only input and output buffers, or processes
+ * under a fixed device-memory cap that must not grow (or synchronise the device through an
+ * allocation) while serving.
+ *
+ * The activation workspace comes from a static array inside the library, MXQ_NOALLOC_SCRATCH_BYTES
+ * bytes per GPU, held by every GPU that loads the library until the process exits.  Problems
+ * whose mxq_linear_workspace_size(M, K, fmt) exceeds that size are rejected with
+ * MXQ_ERR_WORKSPACE before anything is launched (8 MiB covers, e.g., up to 2048 tokens at K = 5120
+ * for FP4).  Other arguments, requirements and results are exactly those of mxq_linear; the caller
+ * still provides x, the quantized weights and `out`.  The call allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture.  All calls share the one array
+ * and it keeps the last call's contents (each call rewrites everything it reads), so calls whose
+ * executions overlap on the GPU -- e.g. on two streams without ordering between them -- race.
+ */
+#define MXQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+int mxq_linear_noalloc(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const float* g_W,
+                       const float* g_A, int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule,
+                       mxq_out out_type, void* out, mxq_stream_t stream);
+
 /* Read the device status word that kernels set when a bounded wait gives up (0 = clean).
  * Synchronizes `stream`.  If reset != 0 the word is cleared afterwards. */
 int mxq_device_status(int* status_out, int reset, mxq_stream_t stream);

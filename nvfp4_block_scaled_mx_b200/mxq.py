@@ -34,6 +34,7 @@ SIGNATURES = {
     "mxq_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_linear_workspace_size": (_SZ, [_I64, _I64, _I]),
     "mxq_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _SZ, _P, _P]),
+    "mxq_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
     "mxq_device_status": (_I, [ctypes.POINTER(_I), _I, _P]),
     "mxq_selftest_timeout": (_I, [_U64, _P]),
     "mxq_strerror": (ctypes.c_char_p, [_I]),

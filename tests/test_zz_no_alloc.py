@@ -1,0 +1,71 @@
+"""The allocation-free linear entry point (mxq_linear_noalloc).
+
+Callers that may not allocate device memory (plugins that only receive their input and output
+buffers, processes under a fixed device-memory cap) use mxq_linear_noalloc, which takes the
+activation workspace from a static array inside the library instead of from the caller.  These
+tests call it through the C ABI and check its output against the regular mxq_linear on the same
+inputs, within the GEMM tolerance used by every other parity test, for two calls in a row (the
+second with fewer tokens and different data, so stale scratch contents would show).  This file
+is collected last on purpose: a failure here leaves every other test already run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_scaled_mx_b200 import mxq, synth
+from tests.helpers import FMTS, check_bf16, check_fp32, oracle_quantize
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(x, Wq, Wsf, N, fmt, rule, out, g_w=None, g_a=None):
+    M, K = x.shape
+    ot = mxq.OUT_FP32 if out.dtype == torch.float32 else mxq.OUT_BF16
+    p = lambda t: None if t is None else t.data_ptr()
+    return mxq.lib().mxq_linear_noalloc(p(x), p(Wq), p(Wsf), p(g_w), p(g_a), M, N, K, mxq.FMT[fmt],
+                                        mxq.RULE[rule], ot, p(out), torch.cuda.current_stream().cuda_stream)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_noalloc_matches_linear_two_calls(fmt, out_dtype):
+    N, K = 384, 1024
+    W = synth.random_bf16((N, K), 5, std=0.02).cuda()
+    g_w = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(W)
+    Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w, layout=mxq.SF_SWIZZLED)
+    Wq_ref, Wsf_ref = oracle_quantize(W.cpu(), fmt, "even", float(g_w.item()) if g_w is not None else 1.0)
+    for M, seed in [(200, 11), (37, 12)]:
+        A = synth.random_bf16((M, K), seed).cuda()
+        g_a = None
+        if fmt == "nvfp4":
+            g_a, _ = mxq.global_scale(A)
+        expect = mxq.linear(A, Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+        out = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
+        assert _noalloc(A, Wq, Wsf, N, fmt, "ceil", out, g_w, g_a) == 0
+        torch.cuda.synchronize()
+        # sum_k |a_k b_k| from the oracle sets the tolerance scale
+        gA = float(g_a.item()) if g_a is not None else 1.0
+        gW = float(g_w.item()) if g_w is not None else 1.0
+        Aq, Asf = oracle_quantize(A.cpu(), fmt, "ceil", gA)
+        _, abs_sum = oracle.gemm(Aq, Asf, Wq_ref, Wsf_ref, M, N, K, FMTS[fmt], gA=gA, gB=gW)
+        got, ref = out.double().cpu().numpy(), expect.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        if out_dtype == torch.float32:
+            check_fp32(got, ref, abs_sum, "noalloc vs linear M=%d" % M)
+        else:
+            check_bf16(got, ref, abs_sum, "noalloc vs linear M=%d" % M)
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    M, N, K = 8192, 256, 5120  # needs 21.0 MB + 1.3 MB of workspace, more than the 8 MiB array
+    assert mxq.mxq_linear_workspace_size(M, K, mxq.MXFP4) > (8 << 20)
+    x = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    Wq = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    Wsf = torch.empty(mxq.sf_bytes(N, K, "mxfp4"), dtype=torch.uint8, device="cuda")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(x, Wq, Wsf, N, "mxfp4", "ceil", out) == -5  # MXQ_ERR_WORKSPACE, nothing launched
