@@ -1,14 +1,17 @@
 // gemm.cu -- block-scaled GEMM on the sm_100a tensor cores (tcgen05), out = alpha * dq(A) dq(B)^T.
 //
 // One persistent CTA per SM, warp-specialised:
-//   warp 0      TMA producer: A and B tiles (128-byte K slices, 128B-swizzled) and their
-//               swizzled scale tiles (bulk copies) into a STAGES-deep shared-memory ring;
-//   warp 1      TMEM owner and MMA issuer: copies each stage's scales into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues 4 block-scaled MMAs per stage into an
-//               fp32 accumulator of 128 lanes x BN columns;
-//   warps 2-9   epilogue: tcgen05.ld of the accumulator (two warps per 32-lane sub-partition, each
-//               owning half of the BN columns), alpha scaling, bf16 RNE or fp32 conversion,
-//               stores with M/N tail masking.
+//   warp 0       TMA producer: A and B tiles (128-byte K slices, 128B-swizzled) and their
+//                swizzled scale tiles (bulk copies) into a STAGES-deep shared-memory ring;
+//   warp 1       TMEM owner and MMA issuer: 4 block-scaled MMAs per stage into an fp32
+//                accumulator of 128 lanes x BN columns;
+//   warps 2-9    epilogue: tcgen05.ld of the accumulator (two warps per 32-lane sub-partition, each
+//                owning half of the BN columns), alpha scaling, bf16 RNE or fp32 conversion,
+//                stores with M/N tail masking;
+//   warps 10-13  scale staging: each writes the stage's scale tiles into its own TMEM
+//                sub-partition with tcgen05.st (the layout tcgen05.cp .32x128b.warpx4 would produce).
+//                Keeping the scale writes off the MMA thread keeps its tensor-core queue to MMAs
+//                only; issuing tcgen05.cp from the MMA thread cost ~300 clk per stage on B200.
 // Tiles are 128 x BN (BN = 256 or 128) and walked M-fastest so the CTAs resident at one time
 // share the same few B tiles and all of A through L2.
 //
@@ -28,7 +31,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kSfWarps = 4;
+constexpr int kThreads = (2 + kEpiWarps + kSfWarps) * 32;
 
 template <int KIND>
 struct Fmt;
@@ -71,7 +75,7 @@ struct Cfg {
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    static constexpr int N_BARS = 2 * STAGES + 2 * ACC_STAGES;
+    static constexpr int N_BARS = 3 * STAGES + 2 * ACC_STAGES;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;  // + slack for 1024-byte alignment
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -99,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + STAGES;
-    uint64_t* accf = empty + STAGES;
+    uint64_t* sfready = empty + STAGES;
+    uint64_t* accf = sfready + STAGES;
     uint64_t* acce = accf + C::ACC_STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
 
@@ -110,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sfready[s], kSfWarps);
         }
         for (int a = 0; a < C::ACC_STAGES; ++a) {
             mbar_init(&accf[a], 1);
@@ -130,6 +136,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
 
     const int num_tiles = p.m_tiles * p.n_tiles;
+    auto groups_of = [&](int tile) {
+        const int nt = tile / p.m_tiles;
+        int groups = 0;
+#pragma unroll
+        for (int g = 0; g < C::BGROUPS; ++g) groups += (nt * C::BGROUPS + g < p.b_row_tiles) ? 1 : 0;
+        return groups;
+    };
+
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_a = policy_evict_last();
@@ -139,9 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-                int groups = 0;
-#pragma unroll
-                for (int g = 0; g < C::BGROUPS; ++g) groups += (nt * C::BGROUPS + g < p.b_row_tiles) ? 1 : 0;
+                const int groups = groups_of(tile);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 1)) {
                         ok = false;
@@ -175,29 +187,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int nt = tile / p.m_tiles;
-                int groups = 0;
-#pragma unroll
-                for (int g = 0; g < C::BGROUPS; ++g) groups += (nt * C::BGROUPS + g < p.b_row_tiles) ? 1 : 0;
                 if (!mbar_wait(&acce[acc], acc_phase ^ 1u, p.status, 2)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, p.status, 3)) {
+                    // operands landed (TMA) and the stage's scales sit in its TMEM slot (staging warps)
+                    if (!mbar_wait(&full[stage], phase, p.status, 3) || !mbar_wait(&sfready[stage], phase, p.status, 5)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
                     const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
-                    const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
-                    for (int a = 0; a < atoms; ++a)
-                        tc_cp_scales(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
-                    for (int g = 0; g < groups; ++g)
-                        for (int a = 0; a < atoms; ++a)
-                            tc_cp_scales(sf_col + C::SF_COLS_A + a * (BN / 32) + g * 4,
-                                         smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
                     const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
                     const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
 #pragma unroll
@@ -226,6 +226,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+    } else if (warp >= 2 + kEpiWarps) {
+        // scale staging: lane l of every staging warp holds row l of each 512-byte scale tile
+        // (16 bytes = 4 TMEM columns) and writes it into its own sub-partition, so all four
+        // sub-partitions see the same replicated tile.
+        const int sub = warp & 3;
+        const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                if (!mbar_wait(&full[stage], phase, p.status, 6)) {
+                    ok = false;
+                    break;
+                }
+                uint32_t r[C::SF_COLS_STAGE];
+                const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES) + lane * 16;
+                const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES) + lane * 16;
+#pragma unroll
+                for (int a = 0; a < C::SF_ATOMS; ++a) {
+                    const uint4 v = ld_shared_v4(sfa_s + a * 512);
+                    r[a * 4 + 0] = v.x;
+                    r[a * 4 + 1] = v.y;
+                    r[a * 4 + 2] = v.z;
+                    r[a * 4 + 3] = v.w;
+                }
+#pragma unroll
+                for (int a = 0; a < C::SF_ATOMS; ++a) {
+#pragma unroll
+                    for (int g = 0; g < C::BGROUPS; ++g) {
+                        const uint4 v = ld_shared_v4(sfb_s + (g * C::SF_ATOMS + a) * 512);
+                        const int c = C::SF_COLS_A + a * (BN / 32) + g * 4;
+                        r[c + 0] = v.x;
+                        r[c + 1] = v.y;
+                        r[c + 2] = v.z;
+                        r[c + 3] = v.w;
+                    }
+                }
+                tmem_st_cols<C::SF_COLS_STAGE>(tmem_base + lane_addr + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE, r);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfready[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
     } else {
         constexpr int COLS = BN / 2;  // accumulator columns owned by this warp
         const int sub = warp & 3;     // TMEM sub-partition this warp may read
@@ -243,40 +292,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m = mt * kBM + row;
             const int n0 = nt * BN + col0;
             if constexpr (!OUT_F32) {
-                uint32_t packed[COLS / 2];
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
+                const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
+                // 64 columns per pass: two 32-column TMEM loads, bf16 conversion, then the stores
 #pragma unroll
-                for (int c = 0; c < COLS / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + c * 32, r);
-                    tmem_ld_wait();
+                for (int h = 0; h < COLS / 64; ++h) {
+                    uint32_t packed[32];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
-                        if (KIND == 1) {
-                            lo = __fmul_rn(lo, alpha);
-                            hi = __fmul_rn(hi, alpha);
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + h * 64 + c * 32, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
+                            if (KIND == 1) {
+                                lo = __fmul_rn(lo, alpha);
+                                hi = __fmul_rn(hi, alpha);
+                            }
+                            const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                            packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
                         }
-                        const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                        packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
                     }
-                }
-                // the accumulator is free for the next tile once it sits in registers
-                tc_fence_before();
-                mbar_arrive(&acce[acc]);
-                if (m < p.M) {
-                    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
-                    if (n0 + COLS <= p.N && (p.N & 7) == 0) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + n0);
+                    if (h == COLS / 64 - 1) {
+                        // the accumulator is free for the next tile once all of it sits in registers
+                        tc_fence_before();
+                        mbar_arrive(&acce[acc]);
+                    }
+                    if (m < p.M) {
+                        if (vec) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + n0 + h * 64);
 #pragma unroll
-                        for (int v = 0; v < COLS / 8; ++v)
-                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    } else {
-                        uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
+                                                    packed[4 * v + 3]);
+                        } else {
+                            uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
 #pragma unroll
-                        for (int v = 0; v < COLS / 2; ++v) {
-                            const int n = n0 + 2 * v;
-                            if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
-                            if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                            for (int v = 0; v < 32; ++v) {
+                                const int n = n0 + h * 64 + 2 * v;
+                                if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                            }
                         }
                     }
                 }

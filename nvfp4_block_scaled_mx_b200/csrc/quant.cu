@@ -28,10 +28,16 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t kc, uint32
     return ((row >> 7) * col_tiles + (kc >> 2)) * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + (kc & 3u);
 }
 
+// floor(n / d) for n, d < 2^32 with magic = ceil(2^64 / d) (d > 1): the product's high word is
+// exact because the rounding of the magic adds less than 2^-32 to n / d.
+__device__ __forceinline__ uint32_t div_magic(uint32_t n, uint32_t d, uint64_t magic) {
+    return d == 1 ? n : static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(n), magic));
+}
+
 template <int FMT, int RULE, bool SWZ>
 __device__ __forceinline__ void quantize_chunk(const uint4 v, const int64_t ci, const bool ok, const uint32_t kblocks,
-                                               const uint32_t col_tiles, const float g, uint8_t* __restrict__ q,
-                                               uint8_t* __restrict__ sf) {
+                                               const uint64_t kb_magic, const uint32_t col_tiles, const float g,
+                                               uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     constexpr int BS = (FMT == MXQ_NVFP4) ? 16 : 32;
     constexpr int LPB = BS / 8;
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -96,7 +102,7 @@ __device__ __forceinline__ void quantize_chunk(const uint4 v, const int64_t ci, 
         const uint32_t blk = static_cast<uint32_t>(ci / LPB);
         uint32_t off = blk;
         if constexpr (SWZ) {
-            const uint32_t row = blk / kblocks;
+            const uint32_t row = div_magic(blk, kblocks, kb_magic);
             const uint32_t kc = blk - row * kblocks;
             off = swz_offset(row, kc, col_tiles);
         }
@@ -106,7 +112,8 @@ __device__ __forceinline__ void quantize_chunk(const uint4 v, const int64_t ci, 
 
 template <int FMT, int RULE, bool SWZ>
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __restrict__ x, int64_t n_chunks,
-                                                                 uint32_t kblocks, uint32_t col_tiles,
+                                                                 uint32_t kblocks, uint64_t kb_magic,
+                                                                 uint32_t col_tiles,
                                                                  const float* __restrict__ gptr,
                                                                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
@@ -126,7 +133,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u)
-            quantize_chunk<FMT, RULE, SWZ>(v[u], wbase + lane + u * stride, ok[u], kblocks, col_tiles, g, q, sf);
+            quantize_chunk<FMT, RULE, SWZ>(v[u], wbase + lane + u * stride, ok[u], kblocks, kb_magic, col_tiles, g, q,
+                                           sf);
     }
 }
 
@@ -139,8 +147,11 @@ cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* 
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
+    // ceil(2^64 / kblocks); unused when kblocks == 1
+    const uint64_t kb_magic =
+        kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
     quantize_kernel<FMT, RULE, SWZ><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_chunks, kblocks, col_tiles, g, static_cast<uint8_t*>(q),
+        static_cast<const uint4*>(x), n_chunks, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
         static_cast<uint8_t*>(sf));
     return cudaGetLastError();
 }
