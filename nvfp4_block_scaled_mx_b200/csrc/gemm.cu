@@ -382,6 +382,311 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+//
+// Two CTAs of a cluster on two SMs compute one 256 x 256 tile with cta_group::2 MMAs: CTA r loads
+// A rows [128 r, +128) and B rows [128 r, +128) of the tile, so each SM streams 32 KB of operands
+// per 128-byte K slice instead of 48 KB for a 128 x 256 tile of its own.  Every load of both CTAs
+// (operands, the CTA's own A scale tiles and the scale tiles of all 256 B rows) is a TMA load that
+// completes on the leader's barrier; a scale thread in the leader then copies both CTAs' scale
+// tiles into their TMEM (tcgen05.cp.cta_group::2, each CTA from its own shared memory) and commits
+// to a local barrier, and the MMA thread issues the MMAs.  The only cross-CTA signals per stage are
+// the TMA completions and the MMA commit multicast to both CTAs.
+//   warp 0       TMA producer (both CTAs)
+//   warp 1       TMEM owner (both CTAs); MMA issuer (leader)
+//   warp 2       scale copies into TMEM (leader)
+//   warps 3-10   epilogue (both CTAs): two warps per TMEM sub-partition, 128 columns each
+
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = (3 + kPairEpiWarps) * 32;
+
+template <int KIND, int STAGES>
+struct PairCfg {
+    static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
+    static constexpr int BK = 128 * EPB;
+    static constexpr int KSTEPS = BK / MMA_K;
+    static constexpr int KB_PER_MMA = MMA_K / BS;
+    static constexpr int SF_ATOMS = BK / BS / 4;
+    static constexpr int A_BYTES = 128 * 128;
+    static constexpr int B_BYTES = 128 * 128;
+    static constexpr int SFA_BYTES = SF_ATOMS * 512;
+    static constexpr int SFB_BYTES = 2 * SF_ATOMS * 512;
+    static constexpr int CTA_STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int SF_COLS_A = SF_ATOMS * 4;
+    static constexpr int SF_COLS_B = SF_ATOMS * 8;
+    static constexpr int SF_COLS_STAGE = SF_COLS_A + SF_COLS_B;
+    static constexpr int SF_TMEM_BASE = 256;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(SF_TMEM_BASE + STAGES * SF_COLS_STAGE <= 512, "TMEM budget");
+    static_assert(KSTEPS == 4, "4 MMAs per 128-byte stage");
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int N_BARS = 3 * STAGES + 2;
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int KIND, int STAGES, bool OUT_F32>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
+                     const GemmArgs p) {
+    using C = PairCfg<KIND, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // leader: all loads of both CTAs landed
+    uint64_t* sfready = full + STAGES;                                 // leader: scales copied into both TMEMs
+    uint64_t* empty = sfready + STAGES;                                // both: the stage's MMAs are done
+    uint64_t* accf = empty + STAGES;                                   // both: accumulator ready
+    uint64_t* acce = accf + 1;                                         // leader: accumulator drained by both
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = static_cast<int>(blockIdx.x >> 1), num_pairs = static_cast<int>(gridDim.x >> 1);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_a);
+        prefetch_tmap(&tma_b);
+        prefetch_tmap(&tma_sfa);
+        prefetch_tmap(&tma_sfb);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sfready[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 2 * kPairEpiWarps);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_wait();
+
+    const int m_tiles = (p.M + 255) / 256;
+    const int num_tiles = m_tiles * p.n_tiles;
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();
+            const uint64_t pol_b = policy_evict_normal();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int mt = tile % m_tiles, nt = tile / m_tiles;
+                const int a_tile = 2 * mt + static_cast<int>(rank);  // this CTA's 128-row tile of A
+                const int b_tile = 2 * nt + static_cast<int>(rank);  // this CTA's 128-row tile of B
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::CTA_STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                    tma_load_2d_pair(&tma_a, fb, smem + C::OFF_A + stage * C::A_BYTES, ks * 128, a_tile * 128, pol_a);
+                    tma_load_2d_pair(&tma_b, fb, smem + C::OFF_B + stage * C::B_BYTES, ks * 128, b_tile * 128, pol_b);
+                    // scale tiles: rows of 256 bytes (half a 512-byte tile); a box covers SF_ATOMS tiles
+                    const int kcol = ks * C::SF_ATOMS;
+                    tma_load_2d_pair(&tma_sfa, fb, smem + C::OFF_SFA + stage * C::SFA_BYTES, 0,
+                                     (a_tile * p.sf_col_tiles + kcol) * 2, pol_a);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        tma_load_2d_pair(&tma_sfb, fb, smem + C::OFF_SFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
+                                         0, ((2 * nt + g) * p.sf_col_tiles + kcol) * 2, pol_b);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                if (!mbar_wait(acce, acc_phase ^ 1u, p.status, 12)) break;
+                tc_fence_after();
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait(&sfready[stage], phase, p.status, 13)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+                    const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                    const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+#pragma unroll
+                    for (int j = 0; j < C::KSTEPS; ++j) {
+                        if (ks * C::BK + j * C::MMA_K < p.K) {
+                            const int kb = j * C::KB_PER_MMA;
+                            const int atom = kb >> 2;
+                            const uint32_t idesc = mma_idesc<KIND>(256, 256, static_cast<uint32_t>(kb & 3));
+                            mma_block_scaled_pair<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                                        smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B), idesc,
+                                                        sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * 8,
+                                                        (ks | j) != 0 ? 1u : 0u);
+                        }
+                    }
+                    tc_commit_pair(&empty[stage], 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(accf, 0x3);
+                acc_phase ^= 1u;
+            }
+        }
+    } else if (warp == 2) {
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, p.status, 16)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+                    const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+#pragma unroll
+                    for (int a = 0; a < C::SF_ATOMS; ++a) {
+                        tc_cp_scales_pair(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
+#pragma unroll
+                        for (int g = 0; g < 2; ++g)
+                            tc_cp_scales_pair(sf_col + C::SF_COLS_A + a * 8 + g * 4,
+                                              smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                    }
+                    tc_commit_pair(&sfready[stage], 0x1);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        constexpr int COLS = 128;  // accumulator columns owned by this warp
+        const int sub = warp & 3;
+        const int col0 = ((warp - 3) >> 2) * COLS;
+        const int row = sub * 32 + lane;
+        const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
+        const uint32_t acce_leader = mapa_shared(smem_u32(acce), 0);
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            if (!mbar_wait(accf, acc_phase, p.status, 14)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
+            const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
+            const int n0 = nt * 256 + col0;
+            if constexpr (!OUT_F32) {
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
+                const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
+#pragma unroll
+                for (int h = 0; h < COLS / 64; ++h) {
+                    uint32_t packed[32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + h * 64 + c * 32, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
+                            if (KIND == 1) {
+                                lo = __fmul_rn(lo, alpha);
+                                hi = __fmul_rn(hi, alpha);
+                            }
+                            const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                            packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
+                        }
+                    }
+                    if (h == COLS / 64 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acce_leader);
+                    }
+                    if (m < p.M) {
+                        if (vec) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + n0 + h * 64);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
+                                                    packed[4 * v + 3]);
+                        } else {
+                            uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+#pragma unroll
+                            for (int v = 0; v < 32; ++v) {
+                                const int n = n0 + h * 64 + 2 * v;
+                                if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                            }
+                        }
+                    }
+                }
+            } else {
+                float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(m) * p.N;
+                const bool vec = (p.N & 3) == 0;
+#pragma unroll 1
+                for (int c = 0; c < COLS / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        const int nb = n0 + c * 32;
+                        if (vec && nb + 32 <= p.N) {
+                            float4* dst = reinterpret_cast<float4*>(orow + nb);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                float4 f;
+                                f.x = __fmul_rn(__uint_as_float(r[4 * v]), alpha);
+                                f.y = __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha);
+                                f.z = __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha);
+                                f.w = __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha);
+                                dst[v] = f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (nb + i < p.N) orow[nb + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce_leader);
+            }
+            acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still signal its barriers or use its TMEM
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -445,11 +750,68 @@ int run(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t stream, bo
     return MXQ_OK;
 }
 
+// Swizzled scales as rows of 256 bytes (two per 512-byte tile); a box covers `tiles` tiles.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kblocks, uint32_t tiles) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const uint64_t half_rows = static_cast<uint64_t>(swizzled_sf_bytes(rows, kblocks) / 256);
+    cuuint64_t dims[2] = {256, half_rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, 2 * tiles};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND, int STAGES, bool F32>
+int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t stream, bool pdl) {
+    using C = PairCfg<KIND, STAGES>;
+    auto kern = gemm_pair_kernel<KIND, STAGES, F32>;
+    const int row_bytes = args.K / C::EPB;
+    const int64_t kblocks = args.K / C::BS;
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_map(&ta, A_q, row_bytes, args.M, 128) || !make_map(&tb, B_q, row_bytes, args.N, 128) ||
+        !make_sf_map(&tsa, args.a_sf, args.M, kblocks, C::SF_ATOMS) ||
+        !make_sf_map(&tsb, args.b_sf, args.N, kblocks, C::SF_ATOMS))
+        return MXQ_ERR_CUDA;
+    args.m_tiles = static_cast<int>(ceil_div(args.M, 256));
+    args.n_tiles = static_cast<int>(ceil_div(args.N, 256));
+    args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = static_cast<int64_t>(args.m_tiles) * args.n_tiles;
+    const int64_t max_pairs = sm_count() / 2;
+    const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kPairThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
 template <int KIND, bool F32>
 int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
-    // 256-wide tiles when they still give at least two waves of work, 128-wide otherwise
-    const int64_t tiles256 = ceil_div(args.M, kBM) * ceil_div(args.N, 256);
-    if (tiles256 >= 2 * static_cast<int64_t>(sm_count())) return run<KIND, 256, 4, F32>(A_q, B_q, args, stream, pdl);
+    // More than 128 rows: CTA pairs on 256 x 256 tiles.  Up to 128 rows (decode): one CTA per
+    // 128 x 128 tile, which gives the most CTAs for the weight stream.
+    if (args.M > 128) return run_pair<KIND, (KIND == 1 ? 5 : 6), F32>(A_q, B_q, args, stream, pdl);
     return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);
 }
 
