@@ -294,46 +294,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (!OUT_F32) {
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
                 const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
-                // 64 columns per pass: two 32-column TMEM loads, bf16 conversion, then the stores
+                // drain this warp's columns into registers (two TMEM loads per wait), release the
+                // accumulator, then store: the stores overlap the next tile's mainloop
+                uint32_t packed[COLS / 2];
 #pragma unroll
-                for (int h = 0; h < COLS / 64; ++h) {
-                    uint32_t packed[32];
+                for (int c = 0; c < COLS / 32; c += 2) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r0);
+                    tmem_ld_32x32b_x32(t_row + c * 32 + 32, r1);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(t_row + h * 64 + c * 32, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
-                            if (KIND == 1) {
-                                lo = __fmul_rn(lo, alpha);
-                                hi = __fmul_rn(hi, alpha);
-                            }
-                            const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                            packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
+                    for (int i = 0; i < 16; ++i) {
+                        float lo = __uint_as_float(r0[2 * i]), hi = __uint_as_float(r0[2 * i + 1]);
+                        float lo1 = __uint_as_float(r1[2 * i]), hi1 = __uint_as_float(r1[2 * i + 1]);
+                        if (KIND == 1) {
+                            lo = __fmul_rn(lo, alpha);
+                            hi = __fmul_rn(hi, alpha);
+                            lo1 = __fmul_rn(lo1, alpha);
+                            hi1 = __fmul_rn(hi1, alpha);
                         }
+                        const __nv_bfloat162 b0 = __floats2bfloat162_rn(lo, hi);
+                        const __nv_bfloat162 b1 = __floats2bfloat162_rn(lo1, hi1);
+                        packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b0);
+                        packed[c * 16 + 16 + i] = *reinterpret_cast<const uint32_t*>(&b1);
                     }
-                    if (h == COLS / 64 - 1) {
-                        // the accumulator is free for the next tile once all of it sits in registers
-                        tc_fence_before();
-                        mbar_arrive(&acce[acc]);
-                    }
-                    if (m < p.M) {
-                        if (vec) {
-                            uint4* dst = reinterpret_cast<uint4*>(orow + n0 + h * 64);
+                }
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+                if (m < p.M) {
+                    if (vec) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + n0);
 #pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                                    packed[4 * v + 3]);
-                        } else {
-                            uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+                        for (int v = 0; v < COLS / 8; ++v)
+                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+                        uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
 #pragma unroll
-                            for (int v = 0; v < 32; ++v) {
-                                const int n = n0 + h * 64 + 2 * v;
-                                if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
-                                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
-                            }
+                        for (int v = 0; v < COLS / 2; ++v) {
+                            const int n = n0 + 2 * v;
+                            if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                            if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
                         }
                     }
                 }
@@ -600,45 +600,47 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             if constexpr (!OUT_F32) {
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
                 const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
+                // drain this warp's columns into registers (two TMEM loads per wait), release the
+                // accumulator, then store: the stores overlap the next tile's mainloop
+                uint32_t packed[COLS / 2];
 #pragma unroll
-                for (int h = 0; h < COLS / 64; ++h) {
-                    uint32_t packed[32];
+                for (int c = 0; c < COLS / 32; c += 2) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r0);
+                    tmem_ld_32x32b_x32(t_row + c * 32 + 32, r1);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(t_row + h * 64 + c * 32, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
-                            if (KIND == 1) {
-                                lo = __fmul_rn(lo, alpha);
-                                hi = __fmul_rn(hi, alpha);
-                            }
-                            const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                            packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b);
+                    for (int i = 0; i < 16; ++i) {
+                        float lo = __uint_as_float(r0[2 * i]), hi = __uint_as_float(r0[2 * i + 1]);
+                        float lo1 = __uint_as_float(r1[2 * i]), hi1 = __uint_as_float(r1[2 * i + 1]);
+                        if (KIND == 1) {
+                            lo = __fmul_rn(lo, alpha);
+                            hi = __fmul_rn(hi, alpha);
+                            lo1 = __fmul_rn(lo1, alpha);
+                            hi1 = __fmul_rn(hi1, alpha);
                         }
+                        const __nv_bfloat162 b0 = __floats2bfloat162_rn(lo, hi);
+                        const __nv_bfloat162 b1 = __floats2bfloat162_rn(lo1, hi1);
+                        packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b0);
+                        packed[c * 16 + 16 + i] = *reinterpret_cast<const uint32_t*>(&b1);
                     }
-                    if (h == COLS / 64 - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(acce_leader);
-                    }
-                    if (m < p.M) {
-                        if (vec) {
-                            uint4* dst = reinterpret_cast<uint4*>(orow + n0 + h * 64);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce_leader);
+                if (m < p.M) {
+                    if (vec) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + n0);
 #pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                                    packed[4 * v + 3]);
-                        } else {
-                            uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+                        for (int v = 0; v < COLS / 8; ++v)
+                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+                        uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
 #pragma unroll
-                            for (int v = 0; v < 32; ++v) {
-                                const int n = n0 + h * 64 + 2 * v;
-                                if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
-                                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
-                            }
+                        for (int v = 0; v < COLS / 2; ++v) {
+                            const int n = n0 + 2 * v;
+                            if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                            if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
                         }
                     }
                 }
