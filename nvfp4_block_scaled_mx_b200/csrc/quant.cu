@@ -1,11 +1,10 @@
 // quant.cu -- bf16 -> MXFP4 (EVEN / CEIL), NVFP4 and MXFP8 block quantizer, scale swizzle,
 // NVFP4 global scale, and the bounded-wait self-test kernel.
 //
-// The quantizer is a single streaming pass over x: each thread owns 8 consecutive elements
-// (one 16-byte load); the bs/8 threads of a block reduce the block amax on the bf16 bit patterns
-// with warp shuffles, derive the scale, and write packed codes (4 bytes per thread for FP4,
-// 8 for FP8) plus one scale byte per block, either row-major or directly in the swizzled
-// tensor-core layout.  Loads of one warp cover 512 contiguous bytes; stores 128 (FP4) or 256 bytes.
+// The quantizer is a single streaming pass over x: each thread owns 32 consecutive elements of a
+// row (four 16-byte loads; one MX block or two NVFP4 blocks), takes the block amax on the bf16 bit
+// patterns, derives the scale, and writes 16 (FP4) or 32 (FP8) bytes of packed codes plus one scale
+// byte per block, either row-major or directly in the swizzled tensor-core layout.
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 
@@ -13,7 +12,6 @@ namespace mxq {
 namespace {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     uint4 v;
@@ -34,116 +32,139 @@ __device__ __forceinline__ uint32_t div_magic(uint32_t n, uint32_t d, uint64_t m
     return d == 1 ? n : static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(n), magic));
 }
 
-template <int FMT, int RULE, bool SWZ>
-__device__ __forceinline__ void quantize_chunk(const uint4 v, const int64_t ci, const bool ok, const uint32_t kblocks,
-                                               const uint64_t kb_magic, const uint32_t col_tiles, const float g,
-                                               uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
-    constexpr int BS = (FMT == MXQ_NVFP4) ? 16 : 32;
-    constexpr int LPB = BS / 8;
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    // block amax on |bf16| bit patterns (non-negative floats order like their bits)
-    const uint32_t m2 = __vmaxu2(__vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
-                                 __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
-    uint32_t amax16 = max(m2 & 0xFFFFu, m2 >> 16);
-#pragma unroll
-    for (int off = 1; off < LPB; off <<= 1) amax16 = max(amax16, __shfl_xor_sync(0xFFFFFFFFu, amax16, off));
-    const uint32_t abits = amax16 << 16;
-
-    float f[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-
-    uint32_t scale_byte;
-    if constexpr (FMT == MXQ_NVFP4) {
-        const float amax = __uint_as_float(abits);
-        uint32_t s = 0;
-        if (amax != 0.0f) {
-            const float t = __fdiv_rn(amax, 6.0f);
-            const float u = __fdiv_rn(t, g);
-            s = cvt_e4m3x2(u, 0.0f) & 0xFFu;
-        }
-        const float d = __fmul_rn(e4m3_decode_pos(s), g);
-        uint32_t packed;
-        if (d == 0.0f) {
-            packed = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) packed |= (__float_as_uint(f[i]) >> 31) << (4 * i + 3);
-        } else {
-            const float r = __fdiv_rn(1.0f, d);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], r);
-            packed = cvt_e2m1x8(f);
-        }
-        scale_byte = s;
-        if (ok) reinterpret_cast<uint32_t*>(q)[ci] = packed;
-    } else {
-        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
-        // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
-        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
-        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
-        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
-        e = max(e, -127);
-        const float inv = exp2_neg(e);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], inv);
-        scale_byte = static_cast<uint32_t>(e + 127);
-        if constexpr (FMT == MXQ_MXFP8) {
-            const uint32_t lo = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
-            const uint32_t hi = cvt_e4m3x2(f[4], f[5]) | (cvt_e4m3x2(f[6], f[7]) << 16);
-            if (ok) reinterpret_cast<uint2*>(q)[ci] = make_uint2(lo, hi);
-        } else {
-            if (ok) reinterpret_cast<uint32_t*>(q)[ci] = cvt_e2m1x8(f);
-        }
-    }
-    if (ok && (threadIdx.x % LPB) == 0) {
-        const uint32_t blk = static_cast<uint32_t>(ci / LPB);
-        uint32_t off = blk;
-        if constexpr (SWZ) {
-            const uint32_t row = div_magic(blk, kblocks, kb_magic);
-            const uint32_t kc = blk - row * kblocks;
-            off = swz_offset(row, kc, col_tiles);
-        }
-        sf[off] = static_cast<uint8_t>(scale_byte);
-    }
+// ld.global.nc with L1 allocation: the four 16-byte loads of a thread cover 64 contiguous bytes,
+// so the sector halves one load leaves in L1 serve the next.
+__device__ __forceinline__ uint4 ld_nc(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
 }
 
+__device__ __forceinline__ uint32_t amax_bits16(const uint32_t* w, int n) {
+    // max |bf16| over 2n values held as bf16x2 words, as an fp32 bit pattern
+    uint32_t m = w[0] & 0x7FFF7FFFu;
+    for (int i = 1; i < n; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    return max(m & 0xFFFFu, m >> 16) << 16;
+}
+
+// Scale byte offset of block `blk` (row-major block index) in the requested layout.
+template <bool SWZ>
+__device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks, uint64_t kb_magic, uint32_t col_tiles) {
+    if constexpr (!SWZ) return blk;
+    const uint32_t row = div_magic(blk, kblocks, kb_magic);
+    const uint32_t kc = blk - row * kblocks;
+    return swz_offset(row, kc, col_tiles);
+}
+
+// One thread quantizes 32 consecutive elements of a row: one MX block (MXFP4 / MXFP8) or two
+// NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8) per thread, coalesced across the warp.
 template <int FMT, int RULE, bool SWZ>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __restrict__ x, int64_t n_chunks,
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __restrict__ x, int64_t n_units,
                                                                  uint32_t kblocks, uint64_t kb_magic,
                                                                  uint32_t col_tiles,
                                                                  const float* __restrict__ gptr,
                                                                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
     pdl_launch_dependents();
     const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
-    const int lane = threadIdx.x & 31;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    // warp-uniform loop bound so that every lane takes part in the shuffles
-    for (int64_t wbase = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); wbase < n_chunks;
-         wbase += kQuantUnroll * stride) {
-        uint4 v[kQuantUnroll];
-        bool ok[kQuantUnroll];
+    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
+        uint32_t w[16];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t ci = wbase + lane + u * stride;
-            ok[u] = ci < n_chunks;
-            v[u] = ok[u] ? ld_stream(x + ci) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = ld_nc(x + u * 4 + i);
+            w[4 * i + 0] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
         }
+        if constexpr (FMT == MXQ_NVFP4) {
+            uint32_t codes[4];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u)
-            quantize_chunk<FMT, RULE, SWZ>(v[u], wbase + lane + u * stride, ok[u], kblocks, kb_magic, col_tiles, g, q,
-                                           sf);
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t* wb = w + 8 * b;
+                const float amax = __uint_as_float(amax_bits16(wb, 8));
+                uint32_t s = 0;
+                if (amax != 0.0f) {
+                    const float t = __fdiv_rn(amax, 6.0f);
+                    const float uu = __fdiv_rn(t, g);
+                    s = cvt_e4m3x2(uu, 0.0f) & 0xFFu;
+                }
+                const float d = __fmul_rn(e4m3_decode_pos(s), g);
+                if (d == 0.0f) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t packed = 0;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            packed |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
+                            packed |= (wb[4 * h + i] >> 31) << (8 * i + 7);
+                        }
+                        codes[2 * b + h] = packed;
+                    }
+                } else {
+                    const float r = __fdiv_rn(1.0f, d);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
+                            f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
+                        }
+                        codes[2 * b + h] = cvt_e2m1x8(f);
+                    }
+                }
+                sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
+                    static_cast<uint8_t>(s);
+            }
+            reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        } else {
+            constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
+            // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
+            constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
+            const uint32_t abits = amax_bits16(w, 16);
+            int e = static_cast<int>(abits >> 23) - 127 - EMAX;
+            if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
+            e = max(e, -127);
+            const float inv = exp2_neg(e);
+            if constexpr (FMT == MXQ_MXFP8) {
+                uint32_t codes[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float a0 = __fmul_rn(__uint_as_float(w[2 * i] << 16), inv);
+                    const float a1 = __fmul_rn(__uint_as_float(w[2 * i] & 0xFFFF0000u), inv);
+                    const float b0 = __fmul_rn(__uint_as_float(w[2 * i + 1] << 16), inv);
+                    const float b1 = __fmul_rn(__uint_as_float(w[2 * i + 1] & 0xFFFF0000u), inv);
+                    codes[i] = cvt_e4m3x2(a0, a1) | (cvt_e4m3x2(b0, b1) << 16);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
+                dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            } else {
+                uint32_t codes[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float f[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        f[2 * i] = __fmul_rn(__uint_as_float(w[4 * h + i] << 16), inv);
+                        f[2 * i + 1] = __fmul_rn(__uint_as_float(w[4 * h + i] & 0xFFFF0000u), inv);
+                    }
+                    codes[h] = cvt_e2m1x8(f);
+                }
+                reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            }
+            sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(e + 127);
+        }
     }
 }
 
 template <int FMT, int RULE, bool SWZ>
 cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, cudaStream_t stream) {
-    const int64_t n_chunks = M * K / 8;
+    const int64_t n_units = M * K / 32;
     const uint32_t kblocks = static_cast<uint32_t>(K / block_size(FMT));
     const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
-    int64_t blocks = ceil_div(n_chunks, static_cast<int64_t>(kQuantThreads) * kQuantUnroll);
+    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
@@ -151,7 +172,7 @@ cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* 
     const uint64_t kb_magic =
         kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
     quantize_kernel<FMT, RULE, SWZ><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_chunks, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
+        static_cast<const uint4*>(x), n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
         static_cast<uint8_t*>(sf));
     return cudaGetLastError();
 }
