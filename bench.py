@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--workload", default="prefill_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-others", action="store_true", help="skip the informational other-problem timings")
     ap.add_argument("--M", type=int, default=None, help="override the workload's M (profiling runs)")
     ap.add_argument("--N", type=int, default=None, help="override the workload's N (profiling runs)")
     return ap.parse_args()
@@ -170,6 +171,20 @@ def time_loop(fn, iters, stream):
     return start.elapsed_time(end) / iters / 1e3
 
 
+def time_flushed(fn, iters, stream, flush):
+    """Median device time of fn() with the L2 flushed (a write larger than L2) before each launch."""
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        fn()
+        end.record(stream)
+        end.synchronize()
+        ts.append(start.elapsed_time(end) / 1e3)
+    return sorted(ts)[len(ts) // 2]
+
+
 def run_mxq(args, world, rank, local):
     from nvfp4_block_scaled_mx_b200 import mxq
     if not torch.cuda.is_available():
@@ -226,12 +241,15 @@ def run_mxq(args, world, rank, local):
     a_sf = ws[(qbytes + 255) // 256 * 256:]
     gemm_s = time_loop(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a, g_B=g_w,
                                         out=out, stream=stream), max(10, args.steps // 4), stream)
-    quant_s = time_loop(lambda: mxq.quantize(A, fmt, cfg["a_rule"], global_scale=g_a, layout=mxq.SF_SWIZZLED,
-                                             q_out=a_q, sf_out=a_sf, stream=stream), max(10, args.steps // 4), stream)
+    # the quantizers are timed one launch at a time with the 126 MB L2 flushed before each
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    quant_s = time_flushed(lambda: mxq.quantize(A, fmt, cfg["a_rule"], global_scale=g_a, layout=mxq.SF_SWIZZLED,
+                                                q_out=a_q, sf_out=a_sf, stream=stream), 20, stream, flush)
     tensor_peak = bf16_tflops * (FP8_PER_BF16 if fmt == "mxfp8" else FP4_PER_BF16)
     gemm_tflops = flops / gemm_s / 1e12
-    roofline = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::%s)" % {"mxfp4": "mxf4", "nvfp4": "mxf4nvf4",
-                                                                                 "mxfp8": "mxf8f6f4"}[fmt],
+    kind = {"mxfp4": "mxf4", "nvfp4": "mxf4nvf4", "mxfp8": "mxf8f6f4"}[fmt]
+    roofline = {"bound": "tensor", "kernel": ("gemm_pair_kernel (tcgen05 cta_group::2 kind::%s)" if M > 128 else
+                                              "gemm_kernel (tcgen05 kind::%s)") % kind,
                 "achieved": round(gemm_tflops, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
                 "frac": round(gemm_tflops / tensor_peak, 4),
                 "peak_source": "%s bf16 %.1f TFLOP/s x %g nominal %s:bf16 ratio" % (
@@ -242,11 +260,19 @@ def run_mxq(args, world, rank, local):
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
              "gbs": round(qb / quant_s / 1e9, 1), "frac": round(qb / quant_s / 1e9 / hbm_gbs, 4),
-             "peak_gbs": hbm_gbs, "ms": round(quant_s * 1e3, 4), "algorithmic_bytes": qb}
+             "peak_gbs": hbm_gbs, "ms": round(quant_s * 1e3, 4), "algorithmic_bytes": qb, "l2": "flushed per launch"}
+    fq_out = torch.empty_like(A)
+    fq_s = time_flushed(lambda: mxq.fake_quantize(A, fmt, cfg["a_rule"], global_scale=g_a, out=fq_out, stream=stream),
+                        20, stream, flush)
+    fake_quant = {"workload": "fake quantize (quantize-dequantize to bf16) %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
+                  "gbs": round(4.0 * M * K / fq_s / 1e9, 1), "frac": round(4.0 * M * K / fq_s / 1e9 / hbm_gbs, 4),
+                  "ms": round(fq_s * 1e3, 4), "algorithmic_bytes_per_elem": 4.0, "l2": "flushed per launch"}
+    del fq_out
 
     # weight (RTN, EVEN) quantizer on the 451 MB weight tensor
-    wq_s = time_loop(lambda: mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED, q_out=W_q,
-                                          sf_out=W_sf, stream=stream), 20, stream)
+    wq_s = time_flushed(lambda: mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED,
+                                             q_out=W_q, sf_out=W_sf, stream=stream), 10, stream, flush)
+    del flush
     wb = QUANT_BYTES_PER_ELEM[fmt] * N * K
     quant_w = {"workload": "weight quantize %dx%d %s %s" % (N, K, fmt, cfg["w_rule"]),
                "gbs": round(wb / wq_s / 1e9, 1), "frac": round(wb / wq_s / 1e9 / hbm_gbs, 4), "peak_gbs": hbm_gbs,
@@ -255,6 +281,11 @@ def run_mxq(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(step, A, out, flops, args, stream, world, dev)
+    others = None
+    if not args.no_others and world == 1:
+        del A, W, W_q, W_sf, ws, out
+        torch.cuda.empty_cache()
+        others = other_workloads(stream, bf16_tflops)
 
     res = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
@@ -264,7 +295,43 @@ def run_mxq(args, world, rank, local):
                       "weight_rule": cfg["w_rule"], "out": cfg["out"], "l2": "working set > 126 MB L2, no flush",
                       "parallelism": "replicas x%d (no collective)" % world},
            "gpu_launches": 2 * args.steps, "roofline": roofline, "quantize": quant, "quantize_weight": quant_w,
-           "clocks": clk.summary(), "e2e": e2e}
+           "fake_quantize": fake_quant,
+           "clocks": clk.summary(), "e2e": e2e, "other_workloads": others}
+    return res
+
+
+def other_workloads(stream, bf16_tflops):
+    """mxq_linear on the remaining problems (decode, NVFP4 down-proj, MXFP8 attention, lm_head):
+    device-resident inputs, CUDA events, informational (the headline is the prefill problem)."""
+    from nvfp4_block_scaled_mx_b200 import mxq
+    res = {}
+    for name in ["decode", "down_nvfp4", "attn_mxfp8", "lm_head"]:
+        cfg = synth.CONFIGS[name]
+        M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
+        A, W = synth.make_inputs(name, device="cuda")
+        g_w = g_a = None
+        if fmt == "nvfp4":
+            g_w, _ = mxq.global_scale(W)
+            g_a, _ = mxq.global_scale(A)
+        W_q, W_sf = mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w)
+        del W
+        ws = torch.empty(mxq.mxq_linear_workspace_size(M, K, mxq.FMT[fmt]), dtype=torch.uint8, device="cuda")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        f = lambda: mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], g_W=g_w, g_A=g_a, workspace=ws, out=out,
+                               stream=stream)
+        for _ in range(3):
+            f()
+        iters = 200 if M * N < 1e8 else 30
+        t = time_loop(f, iters, stream)
+        peak = bf16_tflops * (FP8_PER_BF16 if fmt == "mxfp8" else FP4_PER_BF16)
+        r = {"M": M, "N": N, "K": K, "fmt": fmt, "ms": round(t * 1e3, 4), "tflops": round(2.0 * M * N * K / t / 1e12, 1),
+             "frac_of_measured_peak": round(2.0 * M * N * K / t / 1e12 / peak, 4)}
+        if name == "decode":  # weight-stream bound: codes + scales of W per call
+            wbytes = W_q.numel() + W_sf.numel()
+            r["weight_gbs"] = round(wbytes / t / 1e9, 1)
+        res[name] = r
+        del A, W_q, W_sf, ws, out
+        torch.cuda.empty_cache()
     return res
 
 

@@ -82,6 +82,17 @@ int mxq_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule
                  const float* global_scale, void* q_out, void* sf_out, mxq_sf_layout layout,
                  mxq_stream_t stream);
 
+/*
+ * Fake quantization (quantize, then dequantize back to bf16): y = bf16(dq(Q(x))) with exactly the
+ * codes and scales mxq_quantize produces, decoded in the format's precision (MX: elem * 2^e, exact;
+ * NVFP4: fl32(elem * d), d = fl32(dec(s) * g)) and rounded once to bf16 (RNE).  This is the
+ * fake-quantized forward of quantization-aware training, bit-identical to the serving quantizer
+ * ("Qwen3.5-9B-MXFP4-QAD-W4A4-LR1e-5-s3000", "Training mode": W4A4 fake-quant, EVEN weights, CEIL
+ * activations).  x, y: [M, K] bf16 (device); y may be x (in place).  Arguments as mxq_quantize.
+ */
+int mxq_fake_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule rule, const float* global_scale,
+                      void* y_bf16, mxq_stream_t stream);
+
 /* Re-lay row-major scales [rows, kblocks] (device) into the swizzled tensor-core layout
  * (device, mxq_sf_bytes(SWIZZLED) bytes, padding zeroed).  Pure byte permutation. */
 int mxq_swizzle_scales(const uint8_t* sf_rowmajor, int64_t rows, int64_t kblocks, uint8_t* sf_swizzled,

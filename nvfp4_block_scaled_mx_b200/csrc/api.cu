@@ -136,6 +136,18 @@ int mxq_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule
                : MXQ_ERR_CUDA;
 }
 
+int mxq_fake_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule rule, const float* global_scale,
+                      void* y_bf16, mxq_stream_t stream) {
+    // same argument rules as mxq_quantize; y takes the place of the codes (and may equal x)
+    int rc = validate_quant(x_bf16, M, K, fmt, rule, global_scale, y_bf16, y_bf16, MXQ_SF_ROWMAJOR);
+    if (rc != MXQ_OK) return rc;
+    if ((rc = check_device()) != MXQ_OK) return rc;
+    return launch_fake_quantize(x_bf16, M, K, fmt, rule, global_scale, y_bf16, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MXQ_OK
+               : MXQ_ERR_CUDA;
+}
+
 int mxq_swizzle_scales(const uint8_t* sf_rowmajor, int64_t rows, int64_t kblocks, uint8_t* sf_swizzled,
                        mxq_stream_t stream) {
     if (!sf_rowmajor || !sf_swizzled) return MXQ_ERR_NULL;

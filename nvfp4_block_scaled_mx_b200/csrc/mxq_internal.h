@@ -27,6 +27,9 @@ inline int64_t swizzled_sf_bytes(int64_t rows, int64_t kblocks) {
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q,
                             void* sf, int layout, cudaStream_t stream);
 
+cudaError_t launch_fake_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* y,
+                                 cudaStream_t stream);
+
 cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream);
 
 cudaError_t launch_global_scale(const void* x, int64_t n, float* g_out, float* amax_out, cudaStream_t stream);

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks,
 // One thread quantizes 32 consecutive elements of a row: one MX block (MXFP4 / MXFP8) or two
 // NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8) per thread, coalesced across the warp.
 template <int FMT, int RULE, bool SWZ>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __restrict__ x, int64_t n_units,
+__global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4* __restrict__ x, int64_t n_units,
                                                                  uint32_t kblocks, uint64_t kb_magic,
                                                                  uint32_t col_tiles,
                                                                  const float* __restrict__ gptr,
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint4* __
                         codes[2 * b + h] = packed;
                     }
                 } else {
-                    const float r = __fdiv_rn(1.0f, d);
+                    const float r = __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         float f[8];
@@ -177,6 +177,128 @@ cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ fake quantization
+
+__device__ __forceinline__ float e2m1_decode(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e == 0 ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
+    return (c & 8u) ? -mag : mag;
+}
+
+__device__ __forceinline__ float e4m3_decode(uint32_t c) {
+    const float mag = e4m3_decode_pos(c & 0x7Fu);
+    return (c & 0x80u) ? -mag : mag;
+}
+
+// 2^e as fp32 for e in [-127, 126] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float exp2_pos(int e) {
+    return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// One thread fake-quantizes 32 consecutive elements: the same codes and scales as quantize_kernel,
+// decoded in the format's precision (MX: elem * 2^e, NVFP4: fl(elem * d)) and rounded once to bf16.
+template <int FMT, int RULE>
+__global__ void __launch_bounds__(kQuantThreads) fake_quantize_kernel(const uint4* x, int64_t n_units,
+                                                                         const float* __restrict__ gptr, uint4* y) {
+    const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = ld_nc(x + u * 4 + i);
+            w[4 * i + 0] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+        }
+        if constexpr (FMT == MXQ_NVFP4) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t* wb = w + 8 * b;
+                const float amax = __uint_as_float(amax_bits16(wb, 8));
+                uint32_t s = 0;
+                if (amax != 0.0f) s = cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), g), 0.0f) & 0xFFu;
+                const float d = __fmul_rn(e4m3_decode_pos(s), g);
+                const float r = d == 0.0f ? 0.0f : __frcp_rn(d);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t codes;
+                    if (d == 0.0f) {
+                        codes = 0;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            codes |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
+                            codes |= (wb[4 * h + i] >> 31) << (8 * i + 7);
+                        }
+                    } else {
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
+                            f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
+                        }
+                        codes = cvt_e2m1x8(f);
+                    }
+                    uint32_t o[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes >> (8 * i)), d),
+                                           __fmul_rn(e2m1_decode(codes >> (8 * i + 4)), d));
+                    y[u * 4 + 2 * b + h] = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        } else {
+            constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
+            constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
+            const uint32_t abits = amax_bits16(w, 16);
+            int e = static_cast<int>(abits >> 23) - 127 - EMAX;
+            if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
+            e = max(e, -127);
+            const float inv = exp2_neg(e), sc = exp2_pos(e);
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+                const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+                uint32_t& oi = o[i & 3];
+                float dlo, dhi;
+                if constexpr (FMT == MXQ_MXFP8) {
+                    const uint32_t c = cvt_e4m3x2(lo, hi);
+                    dlo = e4m3_decode(c & 0xFFu);
+                    dhi = e4m3_decode(c >> 8);
+                } else {
+                    uint16_t c8;
+                    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u16.u8 %0, b;\n\t}\n"
+                        : "=h"(c8)
+                        : "f"(lo), "f"(hi));
+                    dlo = e2m1_decode(c8 & 0xFu);
+                    dhi = e2m1_decode(c8 >> 4);
+                }
+                oi = pack_bf16x2(__fmul_rn(dlo, sc), __fmul_rn(dhi, sc));
+                if ((i & 3) == 3) y[u * 4 + (i >> 2)] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+}
+
+template <int FMT, int RULE>
+cudaError_t launch_fq(const void* x, int64_t M, int64_t K, const float* g, void* y, cudaStream_t stream) {
+    const int64_t n_units = M * K / 32;
+    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    fake_quantize_kernel<FMT, RULE><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), n_units, g, static_cast<uint4*>(y));
+    return cudaGetLastError();
+}
+
 template <bool SWZ>
 cudaError_t launch_q_layout(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q, void* sf,
                             cudaStream_t stream) {
@@ -248,6 +370,16 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int ru
         return launch_q_layout<true>(x, M, K, fmt, rule, g, q, sf, stream);
     }
     return launch_q_layout<false>(x, M, K, fmt, rule, g, q, sf, stream);
+}
+
+cudaError_t launch_fake_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* y,
+                                 cudaStream_t stream) {
+    if (fmt == MXQ_NVFP4) return launch_fq<MXQ_NVFP4, 0>(x, M, K, g, y, stream);
+    if (fmt == MXQ_MXFP8)
+        return rule == MXQ_RULE_CEIL ? launch_fq<MXQ_MXFP8, MXQ_RULE_CEIL>(x, M, K, g, y, stream)
+                                     : launch_fq<MXQ_MXFP8, MXQ_RULE_EVEN>(x, M, K, g, y, stream);
+    return rule == MXQ_RULE_CEIL ? launch_fq<MXQ_MXFP4, MXQ_RULE_CEIL>(x, M, K, g, y, stream)
+                                 : launch_fq<MXQ_MXFP4, MXQ_RULE_EVEN>(x, M, K, g, y, stream);
 }
 
 cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream) {

@@ -29,6 +29,7 @@ SIGNATURES = {
     "mxq_q_bytes": (_I, [_I64, _I64, _I, ctypes.POINTER(_SZ)]),
     "mxq_sf_bytes": (_I, [_I64, _I64, _I, _I, ctypes.POINTER(_SZ)]),
     "mxq_quantize": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P, _I, _P]),
+    "mxq_fake_quantize": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P]),
     "mxq_swizzle_scales": (_I, [_P, _I64, _I64, _P, _P]),
     "mxq_global_scale": (_I, [_P, _I64, _P, _P, _P]),
     "mxq_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
@@ -97,6 +98,10 @@ def mxq_quantize(x, M, K, fmt, rule, global_scale, q_out, sf_out, layout, stream
     return lib().mxq_quantize(x, M, K, fmt, rule, global_scale, q_out, sf_out, layout, stream)
 
 
+def mxq_fake_quantize(x, M, K, fmt, rule, global_scale, y, stream):
+    return lib().mxq_fake_quantize(x, M, K, fmt, rule, global_scale, y, stream)
+
+
 def mxq_swizzle_scales(sf_rowmajor, rows, kblocks, sf_swizzled, stream):
     return lib().mxq_swizzle_scales(sf_rowmajor, rows, kblocks, sf_swizzled, stream)
 
@@ -158,6 +163,16 @@ def quantize(x, fmt, rule=EVEN, global_scale=None, layout=SF_SWIZZLED, q_out=Non
     _check(mxq_quantize(_ptr(x), M, K, f, r, _ptr(global_scale), _ptr(q_out), _ptr(sf_out), layout,
                         _stream(stream)), "mxq_quantize")
     return q_out, sf_out
+
+
+def fake_quantize(x, fmt, rule=EVEN, global_scale=None, out=None, stream=None):
+    """x [M, K] bf16 (CUDA) -> bf16 quantize-dequantize of x (out may be x for in-place)."""
+    M, K = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(mxq_fake_quantize(_ptr(x), M, K, _fmt(fmt), _rule(rule), _ptr(global_scale), _ptr(out), _stream(stream)),
+           "mxq_fake_quantize")
+    return out
 
 
 def swizzle_scales(sf_rowmajor, out=None, stream=None):

@@ -323,3 +323,58 @@ int orc_gemm(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Bq, const uin
     free(brow);
     return 0;
 }
+
+/* ---------------------------------------------------------------- fake quantization */
+
+/* fp32 -> bf16 bit pattern with round to nearest, ties to even (finite inputs; overflow -> inf). */
+uint16_t orc_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t r = u + 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(r >> 16);
+}
+
+/* Quantize-then-dequantize x[rows][K] (bf16) into bf16 out[rows][K] -- the fake-quantized forward
+ * of quantization-aware training ("Qwen3.5-9B-MXFP4-QAD-W4A4-LR1e-5-s3000", "Training mode": the
+ * training fake-quant is bit-identical to the serving quantizer).  Each element is decoded in its
+ * format's own precision and rounded once to bf16:
+ *   MX:    v = elem * 2^e, exact in fp64, then fp32 (exact unless it overflows) and bf16 RNE;
+ *   NVFP4: v = fl32(elem * d) with d = fl32(dec(s) * g), the same d the encoder used, then bf16 RNE.
+ * Returns 0, or -1 if K is not a multiple of the block size or memory runs out. */
+int orc_fake_quantize(const uint16_t* x, int64_t rows, int64_t K, int fmt, int rule, float g, uint16_t* out) {
+    int bs = fmt_block(fmt);
+    if (K % bs != 0) return -1;
+    int64_t qrow = fmt == ORC_MXFP8 ? K : K / 2;
+    uint8_t* q = (uint8_t*)malloc((size_t)(rows * qrow));
+    uint8_t* sf = (uint8_t*)malloc((size_t)(rows * (K / bs)));
+    if (!q || !sf) {
+        free(q);
+        free(sf);
+        return -1;
+    }
+    memset(q, 0, (size_t)(rows * qrow));
+    orc_quantize(x, rows, K, fmt, rule, g, q, sf);
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t k = 0; k < K; k++) {
+            uint8_t s = sf[r * (K / bs) + k / bs];
+            double elem;
+            if (fmt == ORC_MXFP8) {
+                elem = orc_e4m3_value(q[r * K + k]);
+            } else {
+                uint8_t byte = q[(r * K + k) / 2];
+                elem = orc_e2m1_value(k % 2 == 0 ? (byte & 0xFu) : (byte >> 4));
+            }
+            float v;
+            if (fmt == ORC_NVFP4) {
+                volatile float d = (float)orc_e4m3_value(s) * g;
+                volatile float prod = (float)elem * d;
+                v = prod;
+            } else {
+                v = (float)(elem * orc_e8m0_value(s));
+            }
+            out[r * K + k] = orc_f32_to_bf16(v);
+        }
+    free(q);
+    free(sf);
+    return 0;
+}

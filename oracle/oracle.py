@@ -50,6 +50,8 @@ def lib():
         L.orc_global_scale.argtypes, L.orc_global_scale.restype = [p, i64, p], f
         L.orc_gemm.argtypes = [p, p, p, p, d, d, i64, i64, i64, i32, p, i64, p, i64, p, p]
         L.orc_gemm.restype = i32
+        L.orc_f32_to_bf16.argtypes, L.orc_f32_to_bf16.restype = [f], ctypes.c_uint16
+        L.orc_fake_quantize.argtypes, L.orc_fake_quantize.restype = [p, i64, i64, i32, i32, f, p], i32
         _lib = L
     return _lib
 
@@ -173,3 +175,18 @@ def gemm(Aq, Asf, Bq, Bsf, M, N, K, fmt, gA=1.0, gB=1.0, rows=None, cols=None):
     if rc != 0:
         raise MemoryError("oracle gemm allocation failed")
     return out, absout
+
+
+def f32_to_bf16(v):
+    return lib().orc_f32_to_bf16(float(v))
+
+
+def fake_quantize(x, fmt, rule=EVEN, g=1.0):
+    """Quantize-dequantize x [rows, K] bf16 -> bf16 bit patterns (uint16) of the same shape."""
+    xb = _bits(x)
+    rows, K = xb.shape
+    out = np.zeros((rows, K), dtype=np.uint16)
+    rc = lib().orc_fake_quantize(_ptr(xb), rows, K, fmt, rule, float(g), _ptr(out))
+    if rc != 0:
+        raise ValueError("K=%d is not a multiple of the block size" % K)
+    return out

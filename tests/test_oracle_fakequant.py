@@ -1,0 +1,54 @@
+"""Pins of the oracle's fake quantization (quantize-dequantize to bf16)."""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_block_scaled_mx_b200 import synth
+from tests.test_oracle_quant import _adversarial_bf16
+
+
+def test_f32_to_bf16_matches_torch(orc):
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.standard_normal(20000) * np.exp(rng.uniform(-80, 80, 20000)),
+                        np.array([0.0, -0.0, 1.0, 3.0e38, 1e-40, -1e-44, 1.00390625, 1.01171875])]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([orc.f32_to_bf16(float(a)) for a in v], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fmt,rule", [("mxfp4", "even"), ("mxfp4", "ceil"), ("mxfp8", "even"), ("mxfp8", "ceil"),
+                                      ("nvfp4", "even")])
+def test_fake_quantize_equals_dequantized_codes(orc, fmt, rule):
+    f = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}[fmt]
+    r = orc.EVEN if rule == "even" else orc.CEIL
+    bs = 16 if fmt == "nvfp4" else 32
+    x = _adversarial_bf16(24, 320, 17, huge=3.0e30 if fmt != "nvfp4" else 3.0e6, bs=bs)
+    g = 1.0
+    if fmt == "nvfp4":
+        g, _ = orc.global_scale(x)
+    y = orc.fake_quantize(x, f, r, g=float(g))
+    q, sf = orc.quantize(x, f, r, g=float(g))
+    d = orc.dequantize(q, sf, 320, f, g=float(g))  # fp64 value of each dequantized element
+    yv = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).double().numpy()
+    if fmt == "nvfp4":
+        # one fp32 product then one bf16 rounding: within half a bf16 ulp of the exact q*s*g, plus
+        # the two fp32 roundings
+        assert np.all(np.abs(yv - d) <= np.abs(d) * (2.0 ** -8 + 2.0 ** -22))
+    else:
+        # MX values have at most 4 significant bits: exactly representable in bf16
+        assert np.array_equal(yv, d)
+    # idempotent: fake-quantizing the fake-quantized tensor changes no value (value idempotence)
+    xy = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16)
+    if fmt != "nvfp4":
+        y2 = orc.fake_quantize(xy, f, r, g=float(g))
+        assert np.array_equal(torch.from_numpy(y2.view(np.int16)).view(torch.bfloat16).double().numpy(), yv)
+
+
+def test_fake_quantize_zero_and_sign(orc):
+    x = torch.zeros(2, 32, dtype=torch.bfloat16)
+    x[1] = -0.0
+    x[1, 3] = -0.01  # rounds to -0 after scaling by its own block amax? no: it is the block amax
+    y = orc.fake_quantize(x, orc.MXFP4, orc.CEIL)
+    assert np.all(y[0] == 0)
+    yv = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert yv[1, 3] < 0 and np.all(np.signbit(yv[1]))
