@@ -83,6 +83,17 @@ int mxq_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule
                  mxq_stream_t stream);
 
 /*
+ * NVFP4 quantization with a running-max activation global scale, the observer fused into the
+ * quantizer ("Qwen3.5-27B-NVFP4-GPTQ", Serving-KL table and caveat: the RTN export's running-max
+ * input scales).  The block scales use g = fl(*amax_in / (6 * 448)), the running state from earlier
+ * batches (device fp32[1], positive); in the same pass *amax_out receives max(*amax_in, max |x|),
+ * the state for the next call.  amax_in and amax_out must be different buffers (swap them between
+ * calls).  Other arguments as mxq_quantize with fmt = NVFP4.
+ */
+int mxq_quantize_running(const void* x_bf16, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q_out,
+                         void* sf_out, mxq_sf_layout layout, mxq_stream_t stream);
+
+/*
  * Fake quantization (quantize, then dequantize back to bf16): y = bf16(dq(Q(x))) with exactly the
  * codes and scales mxq_quantize produces, decoded in the format's precision (MX: elem * 2^e, exact;
  * NVFP4: fl32(elem * d), d = fl32(dec(s) * g)) and rounded once to bf16 (RNE).  This is the

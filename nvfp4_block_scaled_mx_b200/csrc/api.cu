@@ -136,6 +136,20 @@ int mxq_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule
                : MXQ_ERR_CUDA;
 }
 
+int mxq_quantize_running(const void* x_bf16, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q_out,
+                         void* sf_out, mxq_sf_layout layout, mxq_stream_t stream) {
+    if (!amax_out) return MXQ_ERR_NULL;
+    int rc = validate_quant(x_bf16, M, K, MXQ_NVFP4, 0, amax_in, q_out, sf_out, layout);
+    if (rc != MXQ_OK) return rc;
+    if (reinterpret_cast<uintptr_t>(amax_out) & 3u) return MXQ_ERR_ALIGN;
+    if (static_cast<const void*>(amax_in) == static_cast<const void*>(amax_out)) return MXQ_ERR_UNSUPPORTED;
+    if ((rc = check_device()) != MXQ_OK) return rc;
+    return launch_quantize_running(x_bf16, M, K, amax_in, amax_out, q_out, sf_out, layout,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MXQ_OK
+               : MXQ_ERR_CUDA;
+}
+
 int mxq_fake_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule rule, const float* global_scale,
                       void* y_bf16, mxq_stream_t stream) {
     // same argument rules as mxq_quantize; y takes the place of the codes (and may equal x)

@@ -92,6 +92,7 @@ struct GemmArgs {
     int b_row_tiles;   // ceil(N / 128)
     int m_tiles, n_tiles, k_stages;
     int* status;
+    uint32_t k_split;  // split-K kernel: CTAs per cluster sharing one output tile
 };
 
 template <int KIND, int BN, int STAGES, bool OUT_F32>
@@ -375,6 +376,233 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ split-K kernel (M <= 128)
+//
+// Few-token problems (decode) have too few 128 x 128 output tiles to keep every SM streaming
+// weights.  Here a cluster of S CTAs shares one output tile, each CTA accumulating a contiguous
+// share of the K stages; the S partial accumulators are reduced through distributed shared memory
+// in the leader (rank 0) CTA, which alone writes the output.  No global workspace is used.
+// Roles are those of gemm_kernel (warp 0 TMA, warp 1 MMA, warps 2-9 epilogue, 10-13 scale staging).
+
+constexpr uint32_t kMaxSplits = 4;
+
+template <int KIND, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_splitk_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                       const GemmArgs p) {
+    constexpr int BN = 128, STAGES = 6;
+    using C = Cfg<KIND, BN, STAGES>;
+    static_assert((kMaxSplits - 1) * 128 * BN * 4 <= STAGES * (C::A_BYTES + C::B_BYTES), "reduction buffer");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* sfready = empty + STAGES;
+    uint64_t* accf = sfready + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t split = cluster_ctarank();
+    const uint32_t splits = p.k_split;
+    const int nt = static_cast<int>(blockIdx.x / splits);
+    const int per = (p.k_stages + static_cast<int>(splits) - 1) / static_cast<int>(splits);
+    const int k0 = static_cast<int>(split) * per;
+    const int k1 = min(p.k_stages, k0 + per);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_a);
+        prefetch_tmap(&tma_b);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&sfready[s], kSfWarps);
+        }
+        mbar_init(accf, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+
+    const bool b_group = nt < p.b_row_tiles;  // always true: one 128-row B group per tile
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int ks = k0; ks < k1; ++ks) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 21)) break;
+                const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
+                mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
+                tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES, ks * 128, 0, pol);
+                tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, nt * BN, pol);
+                const int64_t kcol = static_cast<int64_t>(ks) * C::SF_ATOMS;
+                bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, p.a_sf + kcol * 512, atoms * 512, &full[stage]);
+                if (b_group)
+                    bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES,
+                              p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + kcol) * 512, atoms * 512,
+                              &full[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int ks = k0; ks < k1; ++ks) {
+                if (!mbar_wait(&full[stage], phase, p.status, 23) || !mbar_wait(&sfready[stage], phase, p.status, 25)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+                const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+#pragma unroll
+                for (int j = 0; j < C::KSTEPS; ++j) {
+                    if (ks * C::BK + j * C::MMA_K < p.K) {
+                        const int kb = j * C::KB_PER_MMA;
+                        const int atom = kb >> 2;
+                        mma_block_scaled<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               mma_idesc<KIND>(kBM, BN, static_cast<uint32_t>(kb & 3)),
+                                               sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * (BN / 32),
+                                               (ks > k0 || j > 0) ? 1u : 0u);
+                    }
+                }
+                tc_commit(&empty[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit(accf);
+        }
+    } else if (warp >= 2 + kEpiWarps) {
+        const int sub = warp & 3;
+        const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait(&full[stage], phase, p.status, 26)) break;
+            uint32_t r[C::SF_COLS_STAGE];
+            const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES) + lane * 16;
+            const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES) + lane * 16;
+#pragma unroll
+            for (int a = 0; a < C::SF_ATOMS; ++a) {
+                const uint4 va = ld_shared_v4(sfa_s + a * 512);
+                r[a * 4 + 0] = va.x;
+                r[a * 4 + 1] = va.y;
+                r[a * 4 + 2] = va.z;
+                r[a * 4 + 3] = va.w;
+                const uint4 vb = ld_shared_v4(sfb_s + a * 512);
+                r[C::SF_COLS_A + a * 4 + 0] = vb.x;
+                r[C::SF_COLS_A + a * 4 + 1] = vb.y;
+                r[C::SF_COLS_A + a * 4 + 2] = vb.z;
+                r[C::SF_COLS_A + a * 4 + 3] = vb.w;
+            }
+            tmem_st_cols<C::SF_COLS_STAGE>(tmem_base + lane_addr + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE, r);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfready[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+
+    // reduction: every CTA's epilogue warps hold their share of the partial tile in registers
+    constexpr int COLS = BN / 2;
+    const bool epi = warp >= 2 && warp < 2 + kEpiWarps;
+    const int sub = warp & 3;
+    const int col0 = ((warp - 2) >> 2) * COLS;
+    const int row = sub * 32 + lane;
+    float acc[COLS];
+    if (epi) {
+        const bool ok = mbar_wait(accf, 0, p.status, 24);
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
+#pragma unroll
+        for (int c = 0; c < COLS / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c * 32 + i] = ok ? __uint_as_float(r[i]) : 0.0f;
+        }
+        tc_fence_before();
+    }
+    // 1: every CTA's MMAs are done, so the leader's operand ring is free for the partials
+    __syncthreads();
+    cluster_sync();
+    float* red = reinterpret_cast<float*>(smem);  // leader: [splits-1][128 rows][BN] fp32
+    if (epi && split != 0 && row < p.M) {
+        const uint32_t dst = mapa_shared(smem_u32(red + ((split - 1) * 128 + row) * BN + col0), 0);
+#pragma unroll
+        for (int v = 0; v < COLS / 4; ++v)
+            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + v * 16), "f"(acc[4 * v]),
+                         "f"(acc[4 * v + 1]), "f"(acc[4 * v + 2]), "f"(acc[4 * v + 3])
+                         : "memory");
+    }
+    // 2: all partials sit in the leader's shared memory
+    cluster_sync();
+    if (epi && split == 0 && row < p.M) {
+        for (uint32_t sp = 1; sp < splits; ++sp) {
+            const float* src = red + ((sp - 1) * 128 + row) * BN + col0;
+#pragma unroll
+            for (int i = 0; i < COLS; ++i) acc[i] = __fadd_rn(acc[i], src[i]);
+        }
+        const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
+        const int n0 = nt * BN + col0;
+        if constexpr (!OUT_F32) {
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.N;
+            uint32_t packed[COLS / 2];
+#pragma unroll
+            for (int i = 0; i < COLS / 2; ++i) {
+                const float lo = KIND == 1 ? __fmul_rn(acc[2 * i], alpha) : acc[2 * i];
+                const float hi = KIND == 1 ? __fmul_rn(acc[2 * i + 1], alpha) : acc[2 * i + 1];
+                const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                packed[i] = *reinterpret_cast<const uint32_t*>(&b);
+            }
+            if (n0 + COLS <= p.N && (p.N & 7) == 0) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + n0);
+#pragma unroll
+                for (int v = 0; v < COLS / 8; ++v)
+                    dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            } else {
+                uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+#pragma unroll
+                for (int v = 0; v < COLS / 2; ++v) {
+                    const int n = n0 + 2 * v;
+                    if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                    if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                }
+            }
+        } else {
+            float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.N;
+#pragma unroll
+            for (int i = 0; i < COLS; ++i)
+                if (n0 + i < p.N) orow[n0 + i] = __fmul_rn(acc[i], alpha);
+        }
+    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -810,10 +1038,62 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
 }
 
 template <int KIND, bool F32>
+int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cudaStream_t stream, bool pdl) {
+    using C = Cfg<KIND, 128, 6>;
+    auto kern = gemm_splitk_kernel<KIND, F32>;
+    const int row_bytes = args.K / C::EPB;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A_q, row_bytes, args.M, kBM) || !make_map(&tb, B_q, row_bytes, args.N, 128)) return MXQ_ERR_CUDA;
+    args.m_tiles = 1;
+    args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
+    args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
+    args.k_split = static_cast<uint32_t>(splits);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(args.n_tiles * splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
+// K splits for a one-row-tile problem: as many as keep every cluster of the grid resident at once
+// (at most 4), each split owning at least one K stage.
+int splitk_count(int64_t N, int64_t K, int bk) {
+    const int64_t n_tiles = ceil_div(N, 128);
+    const int64_t k_stages = ceil_div(K, bk);
+    int64_t s = sm_count() / n_tiles;
+    if (s > static_cast<int64_t>(kMaxSplits)) s = kMaxSplits;
+    if (s > k_stages) s = k_stages;
+    if (s < 2) return 1;
+    const int64_t per = ceil_div(k_stages, s);
+    return static_cast<int>(ceil_div(k_stages, per));
+}
+
+template <int KIND, bool F32>
 int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
     // More than 128 rows: CTA pairs on 256 x 256 tiles.  Up to 128 rows (decode): one CTA per
     // 128 x 128 tile, which gives the most CTAs for the weight stream.
     if (args.M > 128) return run_pair<KIND, (KIND == 1 ? 5 : 6), F32>(A_q, B_q, args, stream, pdl);
+    const int splits = splitk_count(args.N, args.K, Cfg<KIND, 128, 6>::BK);
+    if (splits > 1) return run_splitk<KIND, F32>(A_q, B_q, args, splits, stream, pdl);
     return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);
 }
 

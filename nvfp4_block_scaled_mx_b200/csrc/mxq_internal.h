@@ -27,6 +27,9 @@ inline int64_t swizzled_sf_bytes(int64_t rows, int64_t kblocks) {
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q,
                             void* sf, int layout, cudaStream_t stream);
 
+cudaError_t launch_quantize_running(const void* x, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q,
+                                   void* sf, int layout, cudaStream_t stream);
+
 cudaError_t launch_fake_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* y,
                                  cudaStream_t stream);
 

@@ -58,14 +58,18 @@ __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks,
 
 // One thread quantizes 32 consecutive elements of a row: one MX block (MXFP4 / MXFP8) or two
 // NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8) per thread, coalesced across the warp.
-template <int FMT, int RULE, bool SWZ>
+// OBS (NVFP4 only): gptr is a running amax; g = fl(amax / (6*448)) and the tensor amax of x is
+// folded into *amax_out with one atomicMax per warp.
+template <int FMT, int RULE, bool SWZ, bool OBS = false>
 __global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4* __restrict__ x, int64_t n_units,
                                                                  uint32_t kblocks, uint64_t kb_magic,
                                                                  uint32_t col_tiles,
                                                                  const float* __restrict__ gptr,
-                                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+                                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                                                                 unsigned int* __restrict__ amax_out = nullptr) {
     pdl_launch_dependents();
-    const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
+    const float g = (FMT == MXQ_NVFP4) ? (OBS ? __fdiv_rn(*gptr, 2688.0f) : *gptr) : 1.0f;
+    uint32_t seen = 0;  // largest block amax (fp32 bits) this thread quantized, for OBS
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
         uint32_t w[16];
@@ -83,6 +87,7 @@ __global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4*
             for (int b = 0; b < 2; ++b) {
                 const uint32_t* wb = w + 8 * b;
                 const float amax = __uint_as_float(amax_bits16(wb, 8));
+                if (OBS) seen = max(seen, __float_as_uint(amax));
                 uint32_t s = 0;
                 if (amax != 0.0f) {
                     const float t = __fdiv_rn(amax, 6.0f);
@@ -156,6 +161,10 @@ __global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4*
             }
             sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(e + 127);
         }
+    }
+    if constexpr (OBS) {
+        seen = __reduce_max_sync(0xFFFFFFFFu, seen);
+        if ((threadIdx.x & 31) == 0 && seen != 0) atomicMax(amax_out, seen);
     }
 }
 
@@ -300,6 +309,24 @@ cudaError_t launch_fq(const void* x, int64_t M, int64_t K, const float* g, void*
 }
 
 template <bool SWZ>
+cudaError_t launch_q_running(const void* x, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q,
+                             void* sf, cudaStream_t stream) {
+    const int64_t n_units = M * K / 32;
+    const uint32_t kblocks = static_cast<uint32_t>(K / 16);
+    const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
+    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const uint64_t kb_magic =
+        kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
+    quantize_kernel<MXQ_NVFP4, 0, SWZ, true><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), n_units, kblocks, kb_magic, col_tiles, amax_in, static_cast<uint8_t*>(q),
+        static_cast<uint8_t*>(sf), reinterpret_cast<unsigned int*>(amax_out));
+    return cudaGetLastError();
+}
+
+template <bool SWZ>
 cudaError_t launch_q_layout(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q, void* sf,
                             cudaStream_t stream) {
     if (fmt == MXQ_NVFP4) return launch_q<MXQ_NVFP4, 0, SWZ>(x, M, K, g, q, sf, stream);
@@ -380,6 +407,22 @@ cudaError_t launch_fake_quantize(const void* x, int64_t M, int64_t K, int fmt, i
                                      : launch_fq<MXQ_MXFP8, MXQ_RULE_EVEN>(x, M, K, g, y, stream);
     return rule == MXQ_RULE_CEIL ? launch_fq<MXQ_MXFP4, MXQ_RULE_CEIL>(x, M, K, g, y, stream)
                                  : launch_fq<MXQ_MXFP4, MXQ_RULE_EVEN>(x, M, K, g, y, stream);
+}
+
+cudaError_t launch_quantize_running(const void* x, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q,
+                                   void* sf, int layout, cudaStream_t stream) {
+    // amax_out starts from the running state, then takes this batch's maximum
+    cudaError_t e = cudaMemcpyAsync(amax_out, amax_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+    if (e != cudaSuccess) return e;
+    if (layout == MXQ_SF_SWIZZLED) {
+        const int64_t kb = K / 16;
+        if (M % 128 != 0 || kb % 4 != 0) {
+            e = cudaMemsetAsync(sf, 0, static_cast<size_t>(swizzled_sf_bytes(M, kb)), stream);
+            if (e != cudaSuccess) return e;
+        }
+        return launch_q_running<true>(x, M, K, amax_in, amax_out, q, sf, stream);
+    }
+    return launch_q_running<false>(x, M, K, amax_in, amax_out, q, sf, stream);
 }
 
 cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream) {

@@ -29,6 +29,7 @@ SIGNATURES = {
     "mxq_q_bytes": (_I, [_I64, _I64, _I, ctypes.POINTER(_SZ)]),
     "mxq_sf_bytes": (_I, [_I64, _I64, _I, _I, ctypes.POINTER(_SZ)]),
     "mxq_quantize": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P, _I, _P]),
+    "mxq_quantize_running": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "mxq_fake_quantize": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P]),
     "mxq_swizzle_scales": (_I, [_P, _I64, _I64, _P, _P]),
     "mxq_global_scale": (_I, [_P, _I64, _P, _P, _P]),
@@ -162,6 +163,21 @@ def quantize(x, fmt, rule=EVEN, global_scale=None, layout=SF_SWIZZLED, q_out=Non
             sf_out = torch.empty((M, K // block_size(f)), dtype=torch.uint8, device=x.device)
     _check(mxq_quantize(_ptr(x), M, K, f, r, _ptr(global_scale), _ptr(q_out), _ptr(sf_out), layout,
                         _stream(stream)), "mxq_quantize")
+    return q_out, sf_out
+
+
+def quantize_running(x, amax_in, amax_out, layout=SF_SWIZZLED, q_out=None, sf_out=None, stream=None):
+    """NVFP4 quantize of x with g = amax_in/2688; amax_out <- max(amax_in, max|x|)."""
+    M, K = x.shape
+    if q_out is None:
+        q_out = torch.empty(q_shape(M, K, NVFP4), dtype=torch.uint8, device=x.device)
+    if sf_out is None:
+        if layout == SF_SWIZZLED:
+            sf_out = torch.empty(sf_bytes(M, K, NVFP4, layout), dtype=torch.uint8, device=x.device)
+        else:
+            sf_out = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+    _check(lib().mxq_quantize_running(_ptr(x), M, K, _ptr(amax_in), _ptr(amax_out), _ptr(q_out), _ptr(sf_out), layout,
+                                      _stream(stream)), "mxq_quantize_running")
     return q_out, sf_out
 
 

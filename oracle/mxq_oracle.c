@@ -378,3 +378,16 @@ int orc_fake_quantize(const uint16_t* x, int64_t rows, int64_t K, int fmt, int r
     free(sf);
     return 0;
 }
+
+/* ---------------------------------------------------------------- running-max observer */
+
+/* NVFP4 quantization with a running-max global scale ("Qwen3.5-27B-NVFP4-GPTQ", Serving-KL table:
+ * running-max input scales): g = fl(amax_in / 2688), codes and scales as orc_quantize with that g,
+ * and *amax_out = max(amax_in, max |x|).  Returns orc_quantize's status. */
+int orc_quantize_running(const uint16_t* x, int64_t rows, int64_t K, float amax_in, float* amax_out, uint8_t* q,
+                         uint8_t* sf) {
+    volatile float g = amax_in / 2688.0f;
+    float a = (float)block_amax(x, rows * K);
+    *amax_out = a > amax_in ? a : amax_in;
+    return orc_quantize(x, rows, K, ORC_NVFP4, 0, g, q, sf);
+}

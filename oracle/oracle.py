@@ -52,6 +52,7 @@ def lib():
         L.orc_gemm.restype = i32
         L.orc_f32_to_bf16.argtypes, L.orc_f32_to_bf16.restype = [f], ctypes.c_uint16
         L.orc_fake_quantize.argtypes, L.orc_fake_quantize.restype = [p, i64, i64, i32, i32, f, p], i32
+        L.orc_quantize_running.argtypes, L.orc_quantize_running.restype = [p, i64, i64, f, p, p, p], i32
         _lib = L
     return _lib
 
@@ -190,3 +191,16 @@ def fake_quantize(x, fmt, rule=EVEN, g=1.0):
     if rc != 0:
         raise ValueError("K=%d is not a multiple of the block size" % K)
     return out
+
+
+def quantize_running(x, amax_in):
+    """NVFP4 codes/scales with g = amax_in/2688, and the updated running amax."""
+    xb = _bits(x)
+    rows, K = xb.shape
+    q = np.zeros((rows, K // 2), dtype=np.uint8)
+    sf = np.zeros((rows, K // 16), dtype=np.uint8)
+    out = ctypes.c_float(0.0)
+    rc = lib().orc_quantize_running(_ptr(xb), rows, K, float(amax_in), ctypes.byref(out), _ptr(q), _ptr(sf))
+    if rc != 0:
+        raise ValueError("K=%d is not a multiple of 16" % K)
+    return q, sf, np.float32(out.value)

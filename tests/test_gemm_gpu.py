@@ -35,8 +35,9 @@ def _gpu_gemm(a, w, M, N, K, fmt, out_dtype):
     return out.double().cpu().numpy() if out_dtype == torch.bfloat16 else to_np(out).astype(np.float64)
 
 
+# M <= 128 with several K stages runs the split-K cluster kernel; M > 128 the CTA-pair kernel
 SHAPES = [(1, 1, 64), (16, 256, 256), (128, 128, 128), (200, 300, 320), (129, 520, 1024), (300, 257, 576),
-          (64, 96, 5120), (512, 768, 192)]
+          (64, 96, 5120), (512, 768, 192), (100, 1000, 2048), (128, 4096, 512), (1024, 96, 1024)]
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])

@@ -52,3 +52,18 @@ def test_fake_quantize_zero_and_sign(orc):
     assert np.all(y[0] == 0)
     yv = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).float().numpy()
     assert yv[1, 3] < 0 and np.all(np.signbit(yv[1]))
+
+
+def test_running_max_oracle(orc):
+    x = torch.zeros(2, 32, dtype=torch.bfloat16)
+    x[0, 5] = 5.0
+    q, sf, new = orc.quantize_running(x, 2688.0)  # g = 1
+    qref, sfref = orc.quantize(x, orc.NVFP4, 0, g=1.0)
+    assert new == np.float32(5.0) or new == np.float32(2688.0)
+    assert new == np.float32(2688.0)  # running max keeps the larger state
+    assert np.array_equal(q, qref) and np.array_equal(sf, sfref)
+    q2, sf2, new2 = orc.quantize_running(x, 1.0)
+    assert new2 == np.float32(5.0)
+    g = np.float32(1.0) / np.float32(2688.0)
+    q3, sf3 = orc.quantize(x, orc.NVFP4, 0, g=float(g))
+    assert np.array_equal(q2, q3) and np.array_equal(sf2, sf3)
