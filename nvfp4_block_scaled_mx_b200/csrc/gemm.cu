@@ -92,7 +92,8 @@ struct GemmArgs {
     int b_row_tiles;   // ceil(N / 128)
     int m_tiles, n_tiles, k_stages;
     int* status;
-    uint32_t k_split;  // split-K kernel: CTAs per cluster sharing one output tile
+    uint32_t k_split;      // split-K kernel: CTAs per cluster sharing one output tile
+    uint32_t a_box_bytes;  // split-K kernel: bytes of one A load (rows rounded up to 8, <= 128)
 };
 
 template <int KIND, int BN, int STAGES, bool OUT_F32>
@@ -445,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = k0; ks < k1; ++ks) {
                 if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 21)) break;
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
-                mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
+                // A rows past M are not loaded: they only feed accumulator rows that are never stored
+                mbar_arrive_expect_tx(&full[stage], p.a_box_bytes + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
                 tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES, ks * 128, 0, pol);
                 tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, nt * BN, pol);
                 const int64_t kcol = static_cast<int64_t>(ks) * C::SF_ATOMS;
@@ -1043,7 +1045,9 @@ int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cuda
     auto kern = gemm_splitk_kernel<KIND, F32>;
     const int row_bytes = args.K / C::EPB;
     CUtensorMap ta, tb;
-    if (!make_map(&ta, A_q, row_bytes, args.M, kBM) || !make_map(&tb, B_q, row_bytes, args.N, 128)) return MXQ_ERR_CUDA;
+    const uint32_t a_rows = static_cast<uint32_t>(ceil_div(args.M, 8) * 8);
+    if (!make_map(&ta, A_q, row_bytes, args.M, a_rows) || !make_map(&tb, B_q, row_bytes, args.N, 128)) return MXQ_ERR_CUDA;
+    args.a_box_bytes = a_rows * 128;
     args.m_tiles = 1;
     args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
