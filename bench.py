@@ -305,7 +305,7 @@ def other_workloads(stream, bf16_tflops):
     device-resident inputs, CUDA events, informational (the headline is the prefill problem)."""
     from nvfp4_block_scaled_mx_b200 import mxq
     res = {}
-    for name in ["decode", "down_nvfp4", "attn_mxfp8", "lm_head"]:
+    for name in ["decode", "down_nvfp4", "attn_mxfp8", "lm_head", "in_proj_ba"]:
         cfg = synth.CONFIGS[name]
         M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
         A, W = synth.make_inputs(name, device="cuda")
@@ -329,6 +329,15 @@ def other_workloads(stream, bf16_tflops):
         if name == "decode":  # weight-stream bound: codes + scales of W per call
             wbytes = W_q.numel() + W_sf.numel()
             r["weight_gbs"] = round(wbytes / t / 1e9, 1)
+        if name == "down_nvfp4":  # NVFP4 running-max observer quantizer on the 365 MB activation tensor
+            st_in = torch.tensor([float(mxq.global_scale(A)[1].item())], dtype=torch.float32, device="cuda")
+            st_out = torch.empty(1, dtype=torch.float32, device="cuda")
+            q, sf = mxq.quantize_running(A, st_in, st_out)
+            flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+            tq = time_flushed(lambda: mxq.quantize_running(A, st_in, st_out, q_out=q, sf_out=sf, stream=stream), 10,
+                              stream, flush)
+            r["quantize_running_gbs"] = round(QUANT_BYTES_PER_ELEM["nvfp4"] * M * K / tq / 1e9, 1)
+            del q, sf, flush
         res[name] = r
         del A, W_q, W_sf, ws, out
         torch.cuda.empty_cache()

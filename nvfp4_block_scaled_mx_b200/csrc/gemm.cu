@@ -21,6 +21,7 @@
 // Every stage holds 128 bytes of K per row (256 FP4 or 128 FP8 elements), i.e. 4 MMAs.
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "mxq_device.cuh"
@@ -94,6 +95,7 @@ struct GemmArgs {
     int* status;
     uint32_t k_split;      // split-K kernel: CTAs per cluster sharing one output tile
     uint32_t a_box_bytes;  // split-K kernel: bytes of one A load (rows rounded up to 8, <= 128)
+    uint32_t tma_store;    // pair kernel: bf16 output written through TMA stores (N % 8 == 0)
 };
 
 template <int KIND, int BN, int STAGES, bool OUT_F32>
@@ -653,7 +655,10 @@ struct PairCfg {
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    // epilogue staging for TMA stores: one 32-row x 64-column bf16 tile (4 KB, 128B-swizzled) per warp
+    static constexpr int STG_BYTES = 4096;
+    static constexpr int OFF_STG = ((OFF_SFB + STAGES * SFB_BYTES) + 1023) / 1024 * 1024;
+    static constexpr int OFF_BAR = OFF_STG + kPairEpiWarps * STG_BYTES;
     static constexpr int N_BARS = 3 * STAGES + 2;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
@@ -664,7 +669,7 @@ template <int KIND, int STAGES, bool OUT_F32>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                     const GemmArgs p) {
+                     const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
     using C = PairCfg<KIND, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -858,7 +863,28 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acce_leader);
-                if (m < p.M) {
+                if (p.tma_store) {
+                    // 64 columns at a time: rows into the warp's 128B-swizzled staging tile, then one
+                    // TMA store (clipped at the M / N edges), so the output leaves in full lines
+                    uint8_t* stg = smem + C::OFF_STG + (warp - 3) * C::STG_BYTES;
+#pragma unroll
+                    for (int h = 0; h < COLS / 64; ++h) {
+                        if (lane == 0) bulk_wait_group_read0();
+                        __syncwarp();
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                                make_uint4(packed[h * 32 + 4 * c], packed[h * 32 + 4 * c + 1], packed[h * 32 + 4 * c + 2],
+                                           packed[h * 32 + 4 * c + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        const int ys = mt * 256 + static_cast<int>(rank) * 128 + sub * 32;
+                        if (lane == 0 && ys < p.M && n0 + h * 64 < p.N) {  // boxes wholly past the edge are skipped
+                            tma_store_2d(&tma_out, stg, n0 + h * 64, ys);
+                            bulk_commit_group();
+                        }
+                    }
+                } else if (m < p.M) {
                     if (vec) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + n0);
 #pragma unroll
@@ -910,6 +936,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
     }
 
+    if (warp >= 3 && lane == 0) bulk_wait_group0();  // output stores of this warp have landed
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // no CTA leaves while its peer may still signal its barriers or use its TMEM
@@ -982,6 +1009,19 @@ int run(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t stream, bo
     return MXQ_OK;
 }
 
+// bf16 output [M][N] for TMA stores: boxes of 32 rows x 64 columns (128 bytes), 128B swizzle.
+bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // Swizzled scales as rows of 256 bytes (two per 512-byte tile); a box covers `tiles` tiles.
 bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kblocks, uint32_t tiles) {
     auto enc = encode_fn();
@@ -1002,11 +1042,17 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
     auto kern = gemm_pair_kernel<KIND, STAGES, F32>;
     const int row_bytes = args.K / C::EPB;
     const int64_t kblocks = args.K / C::BS;
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, to;
     if (!make_map(&ta, A_q, row_bytes, args.M, 128) || !make_map(&tb, B_q, row_bytes, args.N, 128) ||
         !make_sf_map(&tsa, args.a_sf, args.M, kblocks, C::SF_ATOMS) ||
         !make_sf_map(&tsb, args.b_sf, args.N, kblocks, C::SF_ATOMS))
         return MXQ_ERR_CUDA;
+    memset(&to, 0, sizeof(to));
+    args.tma_store = 0;
+    if (!F32 && args.N % 8 == 0) {
+        if (!make_out_map(&to, args.out, args.M, args.N)) return MXQ_ERR_CUDA;
+        args.tma_store = 1;
+    }
     args.m_tiles = static_cast<int>(ceil_div(args.M, 256));
     args.n_tiles = static_cast<int>(ceil_div(args.N, 256));
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
@@ -1035,7 +1081,7 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, to, args) != cudaSuccess) return MXQ_ERR_CUDA;
     return MXQ_OK;
 }
 
@@ -1095,7 +1141,7 @@ template <int KIND, bool F32>
 int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
     // More than 128 rows: CTA pairs on 256 x 256 tiles.  Up to 128 rows (decode): one CTA per
     // 128 x 128 tile, which gives the most CTAs for the weight stream.
-    if (args.M > 128) return run_pair<KIND, (KIND == 1 ? 5 : 6), F32>(A_q, B_q, args, stream, pdl);
+    if (args.M > 128) return run_pair<KIND, 5, F32>(A_q, B_q, args, stream, pdl);
     const int splits = splitk_count(args.N, args.K, Cfg<KIND, 128, 6>::BK);
     if (splits > 1) return run_splitk<KIND, F32>(A_q, B_q, args, splits, stream, pdl);
     return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);

@@ -31,6 +31,9 @@ CONFIGS = {
     "lm_head": dict(seed=4, M=2048, N=151936, K=5120, fmt="mxfp4", a_rule="ceil", w_rule="even",
                     out="bf16", a=dict(kind="normal", std=1.0), w=dict(kind="normal", std=0.02),
                     stream=1),
+    # fused in_proj_a/in_proj_b of the linear-attention blocks: N = 48 + 48 = 96 (MXFP8)
+    "in_proj_ba": dict(seed=5, M=8192, N=96, K=5120, fmt="mxfp8", a_rule="even", w_rule="even", out="bf16",
+                       a=dict(kind="normal", std=1.0), w=dict(kind="normal", std=0.02)),
 }
 
 _CHUNK_ROWS = 4096

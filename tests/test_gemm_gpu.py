@@ -160,7 +160,7 @@ def test_bounded_wait_selftest():
     assert int(sf[0, 0]) == 125  # amax 1 -> CEIL e = -2
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill_gate_up", "down_nvfp4", "attn_mxfp8", "lm_head"])
+@pytest.mark.parametrize("name", ["decode", "prefill_gate_up", "down_nvfp4", "attn_mxfp8", "lm_head", "in_proj_ba"])
 def test_linear_full_size_sampled(name):
     """Each full-size problem through mxq_linear in the bench's launch configuration (weights
     quantized on the GPU, activations quantized inside the call); a seeded sample of outputs
