@@ -712,23 +712,25 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int m_tiles = (p.M + 255) / 256;
     const int num_tiles = m_tiles * p.n_tiles;
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_b = policy_evict_normal();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int mt = tile % m_tiles, nt = tile / m_tiles;
-                const int a_tile = 2 * mt + static_cast<int>(rank);  // this CTA's 128-row tile of A
-                const int b_tile = 2 * nt + static_cast<int>(rank);  // this CTA's 128-row tile of B
-                for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 11)) {
-                        ok = false;
-                        break;
-                    }
+        // TMA producer: the whole warp runs the loop; one elected lane issues
+        const uint64_t pol_a = policy_evict_last();
+        const uint64_t pol_b = policy_evict_normal();
+        const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            const int a_tile = 2 * mt + static_cast<int>(rank);  // this CTA's 128-row tile of A
+            const int b_tile = 2 * nt + static_cast<int>(rank);  // this CTA's 128-row tile of B
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 11)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::CTA_STAGE_BYTES);
-                    const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                    const uint32_t fb = full_leader + stage * 8;
                     tma_load_2d_pair(&tma_a, fb, smem + C::OFF_A + stage * C::A_BYTES, ks * 128, a_tile * 128, pol_a);
                     tma_load_2d_pair(&tma_b, fb, smem + C::OFF_B + stage * C::B_BYTES, ks * 128, b_tile * 128, pol_b);
                     // scale tiles: rows of 256 bytes (half a 512-byte tile); a box covers SF_ATOMS tiles
@@ -739,23 +741,25 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     for (int g = 0; g < 2; ++g)
                         tma_load_2d_pair(&tma_sfb, fb, smem + C::OFF_SFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
                                          0, ((2 * nt + g) * p.sf_col_tiles + kcol) * 2, pol_b);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
+            // MMA issuer (leader): the whole warp runs the loop; one elected lane issues
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                if (!mbar_wait(acce, acc_phase ^ 1u, p.status, 12)) break;
+                if (!mbar_wait_warp(acce, acc_phase ^ 1u, p.status, 12)) break;
                 tc_fence_after();
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait(&sfready[stage], phase, p.status, 13)) {
+                    if (!mbar_wait_warp(&sfready[stage], phase, p.status, 13)) {
                         ok = false;
                         break;
                     }
@@ -763,37 +767,42 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
                     const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
                     const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int j = 0; j < C::KSTEPS; ++j) {
-                        if (ks * C::BK + j * C::MMA_K < p.K) {
-                            const int kb = j * C::KB_PER_MMA;
-                            const int atom = kb >> 2;
-                            const uint32_t idesc = mma_idesc<KIND>(256, 256, static_cast<uint32_t>(kb & 3));
-                            mma_block_scaled_pair<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
-                                                        smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B), idesc,
-                                                        sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * 8,
-                                                        (ks | j) != 0 ? 1u : 0u);
+                        for (int j = 0; j < C::KSTEPS; ++j) {
+                            if (ks * C::BK + j * C::MMA_K < p.K) {
+                                const int kb = j * C::KB_PER_MMA;
+                                const int atom = kb >> 2;
+                                const uint32_t idesc = mma_idesc<KIND>(256, 256, static_cast<uint32_t>(kb & 3));
+                                mma_block_scaled_pair<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                                            smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B), idesc,
+                                                            sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * 8,
+                                                            (ks | j) != 0 ? 1u : 0u);
+                            }
                         }
+                        tc_commit_pair(&empty[stage], 0x3);
                     }
-                    tc_commit_pair(&empty[stage], 0x3);
+                    __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair(accf, 0x3);
+                if (elect_one()) tc_commit_pair(accf, 0x3);
+                __syncwarp();
                 acc_phase ^= 1u;
             }
         }
     } else if (warp == 2) {
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
+            // scale copies into both CTAs' TMEM (leader): the whole warp runs the loop; one elected lane issues
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, p.status, 16)) {
+                    if (!mbar_wait_warp(&full[stage], phase, p.status, 16)) {
                         ok = false;
                         break;
                     }
@@ -801,15 +810,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
                     const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
                     const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int a = 0; a < C::SF_ATOMS; ++a) {
-                        tc_cp_scales_pair(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
+                        for (int a = 0; a < C::SF_ATOMS; ++a) {
+                            tc_cp_scales_pair(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
 #pragma unroll
-                        for (int g = 0; g < 2; ++g)
-                            tc_cp_scales_pair(sf_col + C::SF_COLS_A + a * 8 + g * 4,
-                                              smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                            for (int g = 0; g < 2; ++g)
+                                tc_cp_scales_pair(sf_col + C::SF_COLS_A + a * 8 + g * 4,
+                                                  smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                        }
+                        tc_commit_pair(&sfready[stage], 0x1);
                     }
-                    tc_commit_pair(&sfready[stage], 0x1);
+                    __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;

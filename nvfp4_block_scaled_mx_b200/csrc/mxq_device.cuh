@@ -74,6 +74,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     }
 }
 
+// The same wait by every lane of a converged warp, with one decision for the warp: a timeout in
+// any lane aborts all of them, so the warp never splits around a later warp-wide operation.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, int where) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, where));
+}
+
+// True in exactly one lane of a converged warp (elect.sync).  Single-thread issue of TMA and
+// tcgen05 instructions goes through it, so the issuing warp stays converged and warp-uniform
+// addresses and descriptors stay in uniform registers: issuing from a diverged single lane costs
+// about twice as many cycles per instruction.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(p));
+    return p != 0;
+}
+
 // ------------------------------------------------------------------ TMA and bulk copies
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
