@@ -149,20 +149,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_b = policy_evict_normal();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-                const int groups = groups_of(tile);
-                for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 1)) {
-                        ok = false;
-                        break;
-                    }
+        // TMA producer: the whole warp runs the loop; one elected lane issues
+        const uint64_t pol_a = policy_evict_last();
+        const uint64_t pol_b = policy_evict_normal();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+            const int groups = groups_of(tile);
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 1)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
                     const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
                     const uint32_t bytes = C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + groups);
                     mbar_arrive_expect_tx(&full[stage], bytes);
@@ -176,34 +177,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
                                   p.b_sf + (static_cast<int64_t>(nt * C::BGROUPS + g) * p.sf_col_tiles + kcol) * 512,
                                   atoms * 512, &full[stage]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                if (!mbar_wait(&acce[acc], acc_phase ^ 1u, p.status, 2)) break;
+        // MMA issuer: the whole warp runs the loop; one elected lane issues
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1u, p.status, 2)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+            for (int ks = 0; ks < p.k_stages; ++ks) {
+                // operands landed (TMA) and the stage's scales sit in its TMEM slot (staging warps)
+                if (!mbar_wait_warp(&full[stage], phase, p.status, 3) || !mbar_wait_warp(&sfready[stage], phase, p.status, 5)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-                for (int ks = 0; ks < p.k_stages; ++ks) {
-                    // operands landed (TMA) and the stage's scales sit in its TMEM slot (staging warps)
-                    if (!mbar_wait(&full[stage], phase, p.status, 3) || !mbar_wait(&sfready[stage], phase, p.status, 5)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
-                    const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-                    const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+                const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                if (elect_one()) {
 #pragma unroll
                     for (int j = 0; j < C::KSTEPS; ++j) {
                         if (ks * C::BK + j * C::MMA_K < p.K) {
@@ -217,17 +220,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     tc_commit(&empty[stage]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
                 }
-                if (!ok) break;
-                tc_commit(&accf[acc]);
-                if (++acc == C::ACC_STAGES) {
-                    acc = 0;
-                    acc_phase ^= 1u;
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
+            }
+            if (!ok) break;
+            if (elect_one()) tc_commit(&accf[acc]);
+            __syncwarp();
+            if (++acc == C::ACC_STAGES) {
+                acc = 0;
+                acc_phase ^= 1u;
             }
         }
     } else if (warp >= 2 + kEpiWarps) {
@@ -441,12 +446,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const bool b_group = nt < p.b_row_tiles;  // always true: one 128-row B group per tile
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int ks = k0; ks < k1; ++ks) {
-                if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, 21)) break;
+        // TMA producer: the whole warp runs the loop; one elected lane issues
+        const uint64_t pol = policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 21)) break;
+            if (elect_one()) {
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
                 // A rows past M are not loaded: they only feed accumulator rows that are never stored
                 mbar_arrive_expect_tx(&full[stage], p.a_box_bytes + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
@@ -458,26 +464,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES,
                               p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + kcol) * 512, atoms * 512,
                               &full[stage]);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+            }
+            __syncwarp();
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int ks = k0; ks < k1; ++ks) {
-                if (!mbar_wait(&full[stage], phase, p.status, 23) || !mbar_wait(&sfready[stage], phase, p.status, 25)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
-                const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-                const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+        // MMA issuer: the whole warp runs the loop; one elected lane issues
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&full[stage], phase, p.status, 23) || !mbar_wait_warp(&sfready[stage], phase, p.status, 25)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+            const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+            const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+            if (elect_one()) {
 #pragma unroll
                 for (int j = 0; j < C::KSTEPS; ++j) {
                     if (ks * C::BK + j * C::MMA_K < p.K) {
@@ -491,13 +499,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 tc_commit(&empty[stage]);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
             }
-            if (ok) tc_commit(accf);
+            __syncwarp();
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
         }
+        if (ok && elect_one()) tc_commit(accf);
+        __syncwarp();
     } else if (warp >= 2 + kEpiWarps) {
         const int sub = warp & 3;
         const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
