@@ -626,41 +626,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ CTA-pair kernel
 //
-// Two CTAs of a cluster on two SMs compute one 256 x 256 tile with cta_group::2 MMAs: CTA r loads
-// A rows [128 r, +128) and B rows [128 r, +128) of the tile, so each SM streams 32 KB of operands
-// per 128-byte K slice instead of 48 KB for a 128 x 256 tile of its own.  Every load of both CTAs
-// (operands, the CTA's own A scale tiles and the scale tiles of all 256 B rows) is a TMA load that
-// completes on the leader's barrier; a scale thread in the leader then copies both CTAs' scale
-// tiles into their TMEM (tcgen05.cp.cta_group::2, each CTA from its own shared memory) and commits
-// to a local barrier, and the MMA thread issues the MMAs.  The only cross-CTA signals per stage are
-// the TMA completions and the MMA commit multicast to both CTAs.
+// Two CTAs of a cluster on two SMs compute one 256 x BN tile with cta_group::2 MMAs: CTA r loads
+// A rows [128 r, +128) and B rows [BN/2 r, +BN/2) of the tile, so each SM streams 128 rows of A
+// and BN/2 rows of B per 128-byte K slice.  Every load of both CTAs (operands, the CTA's own A
+// scale tiles and the scale tiles of all the tile's B rows) is a TMA load that completes on the
+// leader's barrier; a scale warp in the leader then copies both CTAs' scale tiles into their TMEM
+// (tcgen05.cp.cta_group::2, each CTA from its own shared memory) and commits to a local barrier,
+// and the MMA warp issues the MMAs.  The only cross-CTA signals per stage are the TMA completions
+// and the MMA commit multicast to both CTAs.
+//
+// BN = 256 keeps one accumulator (256 TMEM columns + the scale slots fill the 512), so the
+// tensor pipe idles while the epilogue drains it at every tile boundary.  BN = 192 fits two
+// accumulators (2 x 192 + 5 x 24 scale columns): the epilogue drains one while the MMAs fill the
+// other.  A 192-row tile starts 0 or 64 rows into a 128-row scale tile; the MMA then addresses
+// the B scales 0 or 2 TMEM columns into the two copied scale tiles (32 rows per column).
 //   warp 0       TMA producer (both CTAs)
 //   warp 1       TMEM owner (both CTAs); MMA issuer (leader)
 //   warp 2       scale copies into TMEM (leader)
-//   warps 3-10   epilogue (both CTAs): two warps per TMEM sub-partition, 128 columns each
+//   warps 3-     epilogue (both CTAs): EPI_WARPS / 4 warps per TMEM sub-partition, COLS columns each
+// The single-thread roles run as converged warps that issue through one elected lane.
 
-constexpr int kPairEpiWarps = 8;
-constexpr int kPairThreads = (3 + kPairEpiWarps) * 32;
-
-template <int KIND, int STAGES>
+template <int KIND, int STAGES, int BN>
 struct PairCfg {
+    static_assert(BN == 256 || BN == 192, "pair tile width");
     static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
     static constexpr int BK = 128 * EPB;
     static constexpr int KSTEPS = BK / MMA_K;
     static constexpr int KB_PER_MMA = MMA_K / BS;
     static constexpr int SF_ATOMS = BK / BS / 4;
+    static constexpr int ACC = (BN == 256) ? 1 : 2;    // accumulator buffers
+    static constexpr int B_ROWS = BN / 2;              // B rows per CTA
+    static constexpr int COLS = (BN == 256) ? 128 : 64;  // accumulator columns per epilogue warp
+    static constexpr int EPI_WARPS = 4 * (BN / COLS);
+    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
     static constexpr int A_BYTES = 128 * 128;
-    static constexpr int B_BYTES = 128 * 128;
+    static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int SFA_BYTES = SF_ATOMS * 512;
-    static constexpr int SFB_BYTES = 2 * SF_ATOMS * 512;
+    static constexpr int SFB_BYTES = 2 * SF_ATOMS * 512;  // the tile's B rows lie in two 128-row scale tiles
     static constexpr int CTA_STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int SF_COLS_A = SF_ATOMS * 4;
     static constexpr int SF_COLS_B = SF_ATOMS * 8;
     static constexpr int SF_COLS_STAGE = SF_COLS_A + SF_COLS_B;
-    static constexpr int SF_TMEM_BASE = 256;
+    static constexpr int SF_TMEM_BASE = ACC * BN;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(SF_TMEM_BASE + STAGES * SF_COLS_STAGE <= 512, "TMEM budget");
     static_assert(KSTEPS == 4, "4 MMAs per 128-byte stage");
+    static_assert(B_BYTES % 1024 == 0, "128B-swizzled operand buffers stay 1024-byte aligned");
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
@@ -668,26 +679,26 @@ struct PairCfg {
     // epilogue staging for TMA stores: one 32-row x 64-column bf16 tile (4 KB, 128B-swizzled) per warp
     static constexpr int STG_BYTES = 4096;
     static constexpr int OFF_STG = ((OFF_SFB + STAGES * SFB_BYTES) + 1023) / 1024 * 1024;
-    static constexpr int OFF_BAR = OFF_STG + kPairEpiWarps * STG_BYTES;
-    static constexpr int N_BARS = 3 * STAGES + 2;
+    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
+    static constexpr int N_BARS = 3 * STAGES + 2 * ACC;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int KIND, int STAGES, bool OUT_F32>
-__global__ void __launch_bounds__(kPairThreads, 1)
+template <int KIND, int STAGES, int BN, bool OUT_F32>
+__global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                      const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
-    using C = PairCfg<KIND, STAGES>;
+    using C = PairCfg<KIND, STAGES, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // leader: all loads of both CTAs landed
     uint64_t* sfready = full + STAGES;                                 // leader: scales copied into both TMEMs
     uint64_t* empty = sfready + STAGES;                                // both: the stage's MMAs are done
-    uint64_t* accf = empty + STAGES;                                   // both: accumulator ready
-    uint64_t* acce = accf + 1;                                         // leader: accumulator drained by both
+    uint64_t* accf = empty + STAGES;                                   // both: accumulator buffer ready
+    uint64_t* acce = accf + C::ACC;                                    // leader: accumulator buffer drained by both
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -703,8 +714,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mbar_init(&sfready[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
-        mbar_init(acce, 2 * kPairEpiWarps);
+        for (int a = 0; a < C::ACC; ++a) {
+            mbar_init(&accf[a], 1);
+            mbar_init(&acce[a], 2 * C::EPI_WARPS);
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -731,8 +744,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         bool ok = true;
         for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
-            const int a_tile = 2 * mt + static_cast<int>(rank);  // this CTA's 128-row tile of A
-            const int b_tile = 2 * nt + static_cast<int>(rank);  // this CTA's 128-row tile of B
+            const int a_row = (2 * mt + static_cast<int>(rank)) * 128;            // this CTA's A rows
+            const int b_row = nt * BN + static_cast<int>(rank) * C::B_ROWS;       // this CTA's B rows
+            const int sf_b_tile = (nt * BN) >> 7;  // first 128-row scale tile of the tile's B rows
             for (int ks = 0; ks < p.k_stages; ++ks) {
                 if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 11)) {
                     ok = false;
@@ -741,16 +755,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 if (elect_one()) {
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::CTA_STAGE_BYTES);
                     const uint32_t fb = full_leader + stage * 8;
-                    tma_load_2d_pair(&tma_a, fb, smem + C::OFF_A + stage * C::A_BYTES, ks * 128, a_tile * 128, pol_a);
-                    tma_load_2d_pair(&tma_b, fb, smem + C::OFF_B + stage * C::B_BYTES, ks * 128, b_tile * 128, pol_b);
+                    tma_load_2d_pair(&tma_a, fb, smem + C::OFF_A + stage * C::A_BYTES, ks * 128, a_row, pol_a);
+                    tma_load_2d_pair(&tma_b, fb, smem + C::OFF_B + stage * C::B_BYTES, ks * 128, b_row, pol_b);
                     // scale tiles: rows of 256 bytes (half a 512-byte tile); a box covers SF_ATOMS tiles
                     const int kcol = ks * C::SF_ATOMS;
                     tma_load_2d_pair(&tma_sfa, fb, smem + C::OFF_SFA + stage * C::SFA_BYTES, 0,
-                                     (a_tile * p.sf_col_tiles + kcol) * 2, pol_a);
+                                     ((a_row >> 7) * p.sf_col_tiles + kcol) * 2, pol_a);
 #pragma unroll
                     for (int g = 0; g < 2; ++g)
                         tma_load_2d_pair(&tma_sfb, fb, smem + C::OFF_SFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
-                                         0, ((2 * nt + g) * p.sf_col_tiles + kcol) * 2, pol_b);
+                                         0, ((sf_b_tile + g) * p.sf_col_tiles + kcol) * 2, pol_b);
                 }
                 __syncwarp();
                 if (++stage == STAGES) {
@@ -763,11 +777,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (rank == 0) {
             // MMA issuer (leader): the whole warp runs the loop; one elected lane issues
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                if (!mbar_wait_warp(acce, acc_phase ^ 1u, p.status, 12)) break;
+                const int nt = tile / m_tiles;
+                const uint32_t sfb_shift = static_cast<uint32_t>(((nt * BN) & 127) >> 5);  // 0, or 2 for BN = 192
+                if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1u, p.status, 12)) break;
                 tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
                     if (!mbar_wait_warp(&sfready[stage], phase, p.status, 13)) {
                         ok = false;
@@ -783,10 +802,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                             if (ks * C::BK + j * C::MMA_K < p.K) {
                                 const int kb = j * C::KB_PER_MMA;
                                 const int atom = kb >> 2;
-                                const uint32_t idesc = mma_idesc<KIND>(256, 256, static_cast<uint32_t>(kb & 3));
-                                mma_block_scaled_pair<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                const uint32_t idesc = mma_idesc<KIND>(256, BN, static_cast<uint32_t>(kb & 3));
+                                mma_block_scaled_pair<KIND>(d_tmem, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
                                                             smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B), idesc,
-                                                            sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * 8,
+                                                            sf_col + atom * 4, sf_col + C::SF_COLS_A + atom * 8 + sfb_shift,
                                                             (ks | j) != 0 ? 1u : 0u);
                             }
                         }
@@ -799,9 +818,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     }
                 }
                 if (!ok) break;
-                if (elect_one()) tc_commit_pair(accf, 0x3);
+                if (elect_one()) tc_commit_pair(&accf[acc], 0x3);
                 __syncwarp();
-                acc_phase ^= 1u;
+                if (++acc == C::ACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
             }
         }
     } else if (warp == 2) {
@@ -840,25 +862,27 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             }
         }
     } else {
-        constexpr int COLS = 128;  // accumulator columns owned by this warp
+        constexpr int COLS = C::COLS;  // accumulator columns owned by this warp
         const int sub = warp & 3;
         const int col0 = ((warp - 3) >> 2) * COLS;
         const int row = sub * 32 + lane;
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
-        const uint32_t acce_leader = mapa_shared(smem_u32(acce), 0);
+        int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
-            if (!mbar_wait(accf, acc_phase, p.status, 14)) break;
+            const uint32_t acce_leader = mapa_shared(smem_u32(&acce[acc]), 0);
+            if (!mbar_wait(&accf[acc], acc_phase, p.status, 14)) break;
             tc_fence_after();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
+                                   static_cast<uint32_t>(acc * BN + col0);
             const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
-            const int n0 = nt * 256 + col0;
+            const int n0 = nt * BN + col0;
             if constexpr (!OUT_F32) {
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
                 const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
                 // drain this warp's columns into registers (two TMEM loads per wait), release the
-                // accumulator, then store: the stores overlap the next tile's mainloop
+                // accumulator, then store: the stores overlap the MMAs of the next tile
                 uint32_t packed[COLS / 2];
 #pragma unroll
                 for (int c = 0; c < COLS / 32; c += 2) {
@@ -954,7 +978,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acce_leader);
             }
-            acc_phase ^= 1u;
+            if (++acc == C::ACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
         }
     }
 
@@ -1058,14 +1085,14 @@ bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kblocks
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KIND, int STAGES, bool F32>
+template <int KIND, int STAGES, int BN, bool F32>
 int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t stream, bool pdl) {
-    using C = PairCfg<KIND, STAGES>;
-    auto kern = gemm_pair_kernel<KIND, STAGES, F32>;
+    using C = PairCfg<KIND, STAGES, BN>;
+    auto kern = gemm_pair_kernel<KIND, STAGES, BN, F32>;
     const int row_bytes = args.K / C::EPB;
     const int64_t kblocks = args.K / C::BS;
     CUtensorMap ta, tb, tsa, tsb, to;
-    if (!make_map(&ta, A_q, row_bytes, args.M, 128) || !make_map(&tb, B_q, row_bytes, args.N, 128) ||
+    if (!make_map(&ta, A_q, row_bytes, args.M, 128) || !make_map(&tb, B_q, row_bytes, args.N, C::B_ROWS) ||
         !make_sf_map(&tsa, args.a_sf, args.M, kblocks, C::SF_ATOMS) ||
         !make_sf_map(&tsb, args.b_sf, args.N, kblocks, C::SF_ATOMS))
         return MXQ_ERR_CUDA;
@@ -1076,7 +1103,7 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
         args.tma_store = 1;
     }
     args.m_tiles = static_cast<int>(ceil_div(args.M, 256));
-    args.n_tiles = static_cast<int>(ceil_div(args.N, 256));
+    args.n_tiles = static_cast<int>(ceil_div(args.N, BN));
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1091,7 +1118,7 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
     const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(kPairThreads);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -1163,7 +1190,10 @@ template <int KIND, bool F32>
 int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
     // More than 128 rows: CTA pairs on 256 x 256 tiles.  Up to 128 rows (decode): one CTA per
     // 128 x 128 tile, which gives the most CTAs for the weight stream.
-    if (args.M > 128) return run_pair<KIND, 5, F32>(A_q, B_q, args, stream, pdl);
+    // 256 x 256 pair tiles with one accumulator.  256 x 192 tiles with two accumulators (BN = 192)
+    // remove the drain bubble at tile boundaries but measured slower on the prefill problems: at
+    // 384 tensor-pipe cycles per stage the MMA and scale-copy warps can no longer issue ahead.
+    if (args.M > 128) return run_pair<KIND, 5, 256, F32>(A_q, B_q, args, stream, pdl);
     const int splits = splitk_count(args.N, args.K, Cfg<KIND, 128, 6>::BK);
     if (splits > 1) return run_splitk<KIND, F32>(A_q, B_q, args, splits, stream, pdl);
     return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);
