@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include "mxq.h"
@@ -13,6 +14,9 @@ int* status_ptr();
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// cuTensorMapEncodeTiled from the driver (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -1,10 +1,14 @@
 // quant.cu -- bf16 -> MXFP4 (EVEN / CEIL), NVFP4 and MXFP8 block quantizer, scale swizzle,
 // NVFP4 global scale, and the bounded-wait self-test kernel.
 //
-// The quantizer is a single streaming pass over x: each thread owns 32 consecutive elements of a
-// row (four 16-byte loads; one MX block or two NVFP4 blocks), takes the block amax on the bf16 bit
-// patterns, derives the scale, and writes 16 (FP4) or 32 (FP8) bytes of packed codes plus one scale
-// byte per block, either row-major or directly in the swizzled tensor-core layout.
+// The quantizer is a single streaming pass over x.  x is read as rows of 64 bytes (32 elements:
+// one MX block or two NVFP4 blocks) by TMA, 256 rows per box, into a 4-stage shared-memory ring
+// with a 64-byte swizzle; each thread then owns one 32-element row (its four 16-byte pieces sit in
+// different banks), takes the block amax on the bf16 bit patterns, derives the scale, and writes 16
+// (FP4) or 32 (FP8) bytes of packed codes plus one scale byte per block, either row-major or
+// directly in the swizzled tensor-core layout.
+#include <cstring>
+
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 
@@ -56,110 +60,211 @@ __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks,
     return swz_offset(row, kc, col_tiles);
 }
 
-// One thread quantizes 32 consecutive elements of a row: one MX block (MXFP4 / MXFP8) or two
-// NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8) per thread, coalesced across the warp.
+// One NVFP4 block of 16 elements (8 bf16x2 words): the IEEE fp32 scale sequence t = fl(amax/6),
+// u = fl(t/g), s = E4M3(u) (round to nearest even, saturating), d = fl(dec(s) * g), r = fl(1/d),
+// then the elements fl(x * r) to E2M1.  d and r come from per-code tables (nvfp4_tables); s is at
+// most 0x7E, as u is not negative and saturates to 448.  Writes 8 bytes of codes, returns s.
+template <bool OBS>
+__device__ __forceinline__ uint32_t nvfp4_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
+                                                uint32_t* codes, uint32_t& seen) {
+    const float amax = __uint_as_float(amax_bits16(wb, 8));
+    if (OBS) seen = max(seen, __float_as_uint(amax));
+    uint32_t s = 0;
+    if (amax != 0.0f) {
+        const float t = __fdiv_rn(amax, 6.0f);
+        const float uu = __fdiv_rn(t, g);
+        s = cvt_e4m3x2(uu, 0.0f) & 0xFFu;
+    }
+    const float d = tab_d[s];
+    if (d == 0.0f) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                packed |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
+                packed |= (wb[4 * h + i] >> 31) << (8 * i + 7);
+            }
+            codes[h] = packed;
+        }
+    } else {
+        const float r = tab_r[s];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
+                f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
+            }
+            codes[h] = cvt_e2m1x8(f);
+        }
+    }
+    return s;
+}
+
+// d = fl(dec(s) * g) and r = fl(1/d) (0 where d is 0) for the 128 non-negative E4M3 codes s,
+// filled by the first 128 threads of a CTA.
+__device__ __forceinline__ void nvfp4_tables(float g, float* tab_d, float* tab_r) {
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(e4m3_decode_pos(threadIdx.x), g);
+        tab_d[threadIdx.x] = d;
+        tab_r[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d)
+    }
+}
+
+// Quantize one 32-element row w (16 bf16x2 words) with unit index u: one MX block (MXFP4 / MXFP8)
+// or two NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8), coalesced across the warp.
+template <int FMT, int RULE, bool SWZ, bool OBS>
+__device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u, float g, const float* tab_d,
+                                              const float* tab_r, uint32_t kblocks, uint64_t kb_magic,
+                                              uint32_t col_tiles, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                                              uint32_t& seen) {
+    if constexpr (FMT == MXQ_NVFP4) {
+        uint32_t codes[4];
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const uint32_t s = nvfp4_block<OBS>(w + 8 * b, g, tab_d, tab_r, codes + 2 * b, seen);
+            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
+                static_cast<uint8_t>(s);
+        }
+        reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    } else {
+        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
+        // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
+        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
+        const uint32_t abits = amax_bits16(w, 16);
+        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
+        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
+        e = max(e, -127);
+        const float inv = exp2_neg(e);
+        if constexpr (FMT == MXQ_MXFP8) {
+            uint32_t codes[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a0 = __fmul_rn(__uint_as_float(w[2 * i] << 16), inv);
+                const float a1 = __fmul_rn(__uint_as_float(w[2 * i] & 0xFFFF0000u), inv);
+                const float b0 = __fmul_rn(__uint_as_float(w[2 * i + 1] << 16), inv);
+                const float b1 = __fmul_rn(__uint_as_float(w[2 * i + 1] & 0xFFFF0000u), inv);
+                codes[i] = cvt_e4m3x2(a0, a1) | (cvt_e4m3x2(b0, b1) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        } else {
+            uint32_t codes[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[2 * i] = __fmul_rn(__uint_as_float(w[4 * h + i] << 16), inv);
+                    f[2 * i + 1] = __fmul_rn(__uint_as_float(w[4 * h + i] & 0xFFFF0000u), inv);
+                }
+                codes[h] = cvt_e2m1x8(f);
+            }
+            reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        }
+        sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(e + 127);
+    }
+}
+
+constexpr int kQuantStages = 2;
+constexpr int kQuantRows = 256;                       // 64-byte rows (32 elements) per TMA box, two per thread
+constexpr int kQuantBoxThreads = kQuantRows / 2;
+constexpr int kQuantStageBytes = kQuantRows * 64;     // 16 KB of bf16 per stage
+constexpr int kQuantCtasPerSm = 5;
+// ring, barriers, NVFP4 per-code tables of d and 1/d, and 1024-byte alignment slack
+constexpr int kQuantSmem = kQuantStages * kQuantStageBytes + kQuantStages * 8 + 2 * 128 * 4 + 1024;
+
+// x streams through a 2-stage ring of TMA boxes (256 rows of 64 bytes, 64-byte swizzle) in each of
+// up to 5 CTAs of 128 threads per SM; each CTA takes boxes blockIdx.x, blockIdx.x + gridDim.x, ...
+// and each thread quantizes two rows of a box (two independent dependency chains).  One barrier
+// per box: after it every thread has finished with the previous stage, which thread 0 then refills
+// with the box kQuantStages - 1 ahead.
 // OBS (NVFP4 only): gptr is a running amax; g = fl(amax / (6*448)) and the tensor amax of x is
 // folded into *amax_out with one atomicMax per warp.
 template <int FMT, int RULE, bool SWZ, bool OBS = false>
-__global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4* __restrict__ x, int64_t n_units,
-                                                                 uint32_t kblocks, uint64_t kb_magic,
-                                                                 uint32_t col_tiles,
-                                                                 const float* __restrict__ gptr,
-                                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-                                                                 unsigned int* __restrict__ amax_out = nullptr) {
+__global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
+    quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t n_units, uint32_t kblocks, uint64_t kb_magic,
+                    uint32_t col_tiles, const float* __restrict__ gptr, uint8_t* __restrict__ q,
+                    uint8_t* __restrict__ sf, unsigned int* __restrict__ amax_out, int* status,
+                    const void* __restrict__ x_tail, bool tail) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kQuantStages * kQuantStageBytes);
+    float* tab_d = reinterpret_cast<float*>(full + kQuantStages);
+    float* tab_r = tab_d + 128;
     pdl_launch_dependents();
+    const int64_t n_boxes = (n_units + kQuantRows - 1) / kQuantRows;
+    const int64_t step = gridDim.x;
+    if (threadIdx.x == 0) {
+        if (n_boxes > 0) prefetch_tmap(&tmap_x);
+        for (int st = 0; st < kQuantStages; ++st) mbar_init(&full[st], 1);
+        fence_barrier_init();
+        const uint64_t pol = policy_evict_first();
+        for (int st = 0; st < kQuantStages; ++st) {
+            const int64_t b = blockIdx.x + st * step;
+            if (b >= n_boxes) break;
+            mbar_arrive_expect_tx(&full[st], kQuantStageBytes);
+            tma_load_2d(&tmap_x, &full[st], ring + st * kQuantStageBytes, 0, static_cast<int>(b * kQuantRows), pol);
+        }
+    }
     const float g = (FMT == MXQ_NVFP4) ? (OBS ? __fdiv_rn(*gptr, 2688.0f) : *gptr) : 1.0f;
+    if constexpr (FMT == MXQ_NVFP4) nvfp4_tables(g, tab_d, tab_r);
+    __syncthreads();
     uint32_t seen = 0;  // largest block amax (fp32 bits) this thread quantized, for OBS
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
-        uint32_t w[16];
+    // 64-byte swizzle: 16-byte piece c of row r sits at piece c ^ ((r >> 1) & 3); this thread takes
+    // rows t and t + 128 of each box, which share the same swizzle
+    const uint32_t my_row = smem_u32(ring) + threadIdx.x * 64u;
+    const uint32_t sw = (threadIdx.x >> 1) & 3u;
+    int it = 0;
+    for (int64_t b = blockIdx.x; b < n_boxes; b += step, ++it) {
+        const int st = it % kQuantStages;
+        const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(it / kQuantStages) & 1u, status, 30);
+        // every thread is done with the previous stage and no thread leaves alone on a timeout
+        if (__syncthreads_or(!ok)) break;
+        if (threadIdx.x == 0 && it > 0) {
+            const int prev = (it - 1) % kQuantStages;
+            const int64_t nb = b + (kQuantStages - 1) * step;
+            if (nb < n_boxes) {
+                mbar_arrive_expect_tx(&full[prev], kQuantStageBytes);
+                tma_load_2d(&tmap_x, &full[prev], ring + prev * kQuantStageBytes, 0, static_cast<int>(nb * kQuantRows),
+                            policy_evict_first());
+            }
+        }
+        uint32_t w0[16], w1[16];
+        const uint32_t row = my_row + static_cast<uint32_t>(st * kQuantStageBytes);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint4 v = ld_nc(x + u * 4 + i);
-            w[4 * i + 0] = v.x;
-            w[4 * i + 1] = v.y;
-            w[4 * i + 2] = v.z;
-            w[4 * i + 3] = v.w;
+            const uint32_t piece = (static_cast<uint32_t>(i) ^ sw) << 4;
+            const uint4 v0 = ld_shared_v4(row + piece);
+            const uint4 v1 = ld_shared_v4(row + kQuantBoxThreads * 64 + piece);
+            w0[4 * i + 0] = v0.x;
+            w0[4 * i + 1] = v0.y;
+            w0[4 * i + 2] = v0.z;
+            w0[4 * i + 3] = v0.w;
+            w1[4 * i + 0] = v1.x;
+            w1[4 * i + 1] = v1.y;
+            w1[4 * i + 2] = v1.z;
+            w1[4 * i + 3] = v1.w;
         }
-        if constexpr (FMT == MXQ_NVFP4) {
-            uint32_t codes[4];
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const uint32_t* wb = w + 8 * b;
-                const float amax = __uint_as_float(amax_bits16(wb, 8));
-                if (OBS) seen = max(seen, __float_as_uint(amax));
-                uint32_t s = 0;
-                if (amax != 0.0f) {
-                    const float t = __fdiv_rn(amax, 6.0f);
-                    const float uu = __fdiv_rn(t, g);
-                    s = cvt_e4m3x2(uu, 0.0f) & 0xFFu;
-                }
-                const float d = __fmul_rn(e4m3_decode_pos(s), g);
-                if (d == 0.0f) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t packed = 0;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            packed |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
-                            packed |= (wb[4 * h + i] >> 31) << (8 * i + 7);
-                        }
-                        codes[2 * b + h] = packed;
-                    }
-                } else {
-                    const float r = __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float f[8];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
-                            f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
-                        }
-                        codes[2 * b + h] = cvt_e2m1x8(f);
-                    }
-                }
-                sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
-                    static_cast<uint8_t>(s);
-            }
-            reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        } else {
-            constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
-            // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
-            constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
-            const uint32_t abits = amax_bits16(w, 16);
-            int e = static_cast<int>(abits >> 23) - 127 - EMAX;
-            if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
-            e = max(e, -127);
-            const float inv = exp2_neg(e);
-            if constexpr (FMT == MXQ_MXFP8) {
-                uint32_t codes[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float a0 = __fmul_rn(__uint_as_float(w[2 * i] << 16), inv);
-                    const float a1 = __fmul_rn(__uint_as_float(w[2 * i] & 0xFFFF0000u), inv);
-                    const float b0 = __fmul_rn(__uint_as_float(w[2 * i + 1] << 16), inv);
-                    const float b1 = __fmul_rn(__uint_as_float(w[2 * i + 1] & 0xFFFF0000u), inv);
-                    codes[i] = cvt_e4m3x2(a0, a1) | (cvt_e4m3x2(b0, b1) << 16);
-                }
-                uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
-                dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-            } else {
-                uint32_t codes[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    float f[8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        f[2 * i] = __fmul_rn(__uint_as_float(w[4 * h + i] << 16), inv);
-                        f[2 * i + 1] = __fmul_rn(__uint_as_float(w[4 * h + i] & 0xFFFF0000u), inv);
-                    }
-                    codes[h] = cvt_e2m1x8(f);
-                }
-                reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            }
-            sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(e + 127);
+        const int64_t u = b * kQuantRows + threadIdx.x;
+        if (u < n_units) quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
+        if (u + kQuantBoxThreads < n_units)
+            quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q,
+                                               sf, seen);
+    }
+    if constexpr (FMT == MXQ_NVFP4) {
+        // M * K = 16 (mod 32): the last NVFP4 block is half a 32-element row, quantized from global memory
+        if (tail && blockIdx.x == 0 && threadIdx.x == 0) {
+            const uint4* xt = reinterpret_cast<const uint4*>(x_tail);
+            const uint4 v0 = xt[0], v1 = xt[1];
+            const uint32_t wt[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint32_t codes[2];
+            const uint32_t s = nvfp4_block<OBS>(wt, g, tab_d, tab_r, codes, seen);
+            reinterpret_cast<uint2*>(q)[2 * n_units] = make_uint2(codes[0], codes[1]);
+            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * n_units), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(s);
         }
     }
     if constexpr (OBS) {
@@ -168,22 +273,54 @@ __global__ void __launch_bounds__(kQuantThreads, 8) quantize_kernel(const uint4*
     }
 }
 
-template <int FMT, int RULE, bool SWZ>
-cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, cudaStream_t stream) {
+// x [n_units][64 bytes] as a 2-D byte tensor, boxes of 256 rows, 64-byte swizzle.
+bool make_x_map(CUtensorMap* m, const void* x, int64_t n_units) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(n_units)};
+    cuuint64_t strides[1] = {64};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kQuantRows)};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int RULE, bool SWZ, bool OBS>
+cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, unsigned int* amax_out,
+                         cudaStream_t stream) {
     const int64_t n_units = M * K / 32;
+    const bool tail = (M * K) % 32 != 0;  // NVFP4 only: a last block of 16 elements
     const uint32_t kblocks = static_cast<uint32_t>(K / block_size(FMT));
     const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
-    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    CUtensorMap tmap;
+    if (n_units > 0 && !make_x_map(&tmap, x, n_units)) return cudaErrorInvalidValue;
+    if (n_units == 0) memset(&tmap, 0, sizeof(tmap));
+    auto kern = quantize_kernel<FMT, RULE, SWZ, OBS>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantRows));
+    const int64_t cap = static_cast<int64_t>(sm_count()) * kQuantCtasPerSm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     // ceil(2^64 / kblocks); unused when kblocks == 1
     const uint64_t kb_magic =
         kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
-    quantize_kernel<FMT, RULE, SWZ><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
-        static_cast<uint8_t*>(sf));
+    kern<<<static_cast<unsigned>(blocks), kQuantBoxThreads, kQuantSmem, stream>>>(
+        tmap, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf), amax_out,
+        status_ptr(), static_cast<const uint8_t*>(x) + n_units * 64, tail);
     return cudaGetLastError();
+}
+
+template <int FMT, int RULE, bool SWZ>
+cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, cudaStream_t stream) {
+    return launch_q_tma<FMT, RULE, SWZ, false>(x, M, K, g, q, sf, nullptr, stream);
 }
 
 // ------------------------------------------------------------------ fake quantization
@@ -209,12 +346,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// One NVFP4 block of 16 elements fake-quantized: the codes and scale of nvfp4_block, decoded as
+// fl(elem * d) and rounded to bf16; 32 bytes out.
+__device__ __forceinline__ void nvfp4_fake_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
+                                                 uint4* out) {
+    uint32_t codes[2], seen = 0;
+    const uint32_t s = nvfp4_block<false>(wb, g, tab_d, tab_r, codes, seen);
+    const float d = tab_d[s];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes[h] >> (8 * i)), d), __fmul_rn(e2m1_decode(codes[h] >> (8 * i + 4)), d));
+        out[h] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 // One thread fake-quantizes 32 consecutive elements: the same codes and scales as quantize_kernel,
 // decoded in the format's precision (MX: elem * 2^e, NVFP4: fl(elem * d)) and rounded once to bf16.
 template <int FMT, int RULE>
 __global__ void __launch_bounds__(kQuantThreads) fake_quantize_kernel(const uint4* x, int64_t n_units,
-                                                                         const float* __restrict__ gptr, uint4* y) {
+                                                                         const float* __restrict__ gptr, uint4* y,
+                                                                         bool tail) {
     const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
+    __shared__ float tab_d[128], tab_r[128];
+    if constexpr (FMT == MXQ_NVFP4) {
+        nvfp4_tables(g, tab_d, tab_r);
+        __syncthreads();
+    }
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
         uint32_t w[16];
@@ -228,40 +388,7 @@ __global__ void __launch_bounds__(kQuantThreads) fake_quantize_kernel(const uint
         }
         if constexpr (FMT == MXQ_NVFP4) {
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const uint32_t* wb = w + 8 * b;
-                const float amax = __uint_as_float(amax_bits16(wb, 8));
-                uint32_t s = 0;
-                if (amax != 0.0f) s = cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), g), 0.0f) & 0xFFu;
-                const float d = __fmul_rn(e4m3_decode_pos(s), g);
-                const float r = d == 0.0f ? 0.0f : __frcp_rn(d);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t codes;
-                    if (d == 0.0f) {
-                        codes = 0;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            codes |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
-                            codes |= (wb[4 * h + i] >> 31) << (8 * i + 7);
-                        }
-                    } else {
-                        float f[8];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
-                            f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
-                        }
-                        codes = cvt_e2m1x8(f);
-                    }
-                    uint32_t o[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes >> (8 * i)), d),
-                                           __fmul_rn(e2m1_decode(codes >> (8 * i + 4)), d));
-                    y[u * 4 + 2 * b + h] = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
+            for (int b = 0; b < 2; ++b) nvfp4_fake_block(w + 8 * b, g, tab_d, tab_r, y + u * 4 + 2 * b);
         } else {
             constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
             constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
@@ -294,6 +421,14 @@ __global__ void __launch_bounds__(kQuantThreads) fake_quantize_kernel(const uint
             }
         }
     }
+    if constexpr (FMT == MXQ_NVFP4) {
+        // M * K = 16 (mod 32): the last block is half a 32-element unit
+        if (tail && blockIdx.x == 0 && threadIdx.x == 0) {
+            const uint4 v0 = x[n_units * 4], v1 = x[n_units * 4 + 1];
+            const uint32_t wt[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            nvfp4_fake_block(wt, g, tab_d, tab_r, y + n_units * 4);
+        }
+    }
 }
 
 template <int FMT, int RULE>
@@ -304,26 +439,15 @@ cudaError_t launch_fq(const void* x, int64_t M, int64_t K, const float* g, void*
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     fake_quantize_kernel<FMT, RULE><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_units, g, static_cast<uint4*>(y));
+        static_cast<const uint4*>(x), n_units, g, static_cast<uint4*>(y), (M * K) % 32 != 0);
     return cudaGetLastError();
 }
 
 template <bool SWZ>
 cudaError_t launch_q_running(const void* x, int64_t M, int64_t K, const float* amax_in, float* amax_out, void* q,
                              void* sf, cudaStream_t stream) {
-    const int64_t n_units = M * K / 32;
-    const uint32_t kblocks = static_cast<uint32_t>(K / 16);
-    const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
-    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    const uint64_t kb_magic =
-        kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
-    quantize_kernel<MXQ_NVFP4, 0, SWZ, true><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_units, kblocks, kb_magic, col_tiles, amax_in, static_cast<uint8_t*>(q),
-        static_cast<uint8_t*>(sf), reinterpret_cast<unsigned int*>(amax_out));
-    return cudaGetLastError();
+    return launch_q_tma<MXQ_NVFP4, 0, SWZ, true>(x, M, K, amax_in, q, sf, reinterpret_cast<unsigned int*>(amax_out),
+                                                 stream);
 }
 
 template <bool SWZ>

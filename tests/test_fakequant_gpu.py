@@ -19,10 +19,12 @@ def _bits(t):
 
 
 @pytest.mark.parametrize("fmt,rule", COMBOS)
-@pytest.mark.parametrize("shape", [(1, 32), (37, 320), (130, 1056), (256, 5120)])
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (1, 32), (37, 320), (130, 1056), (256, 5120)])
 def test_fake_quantize_matches_oracle(fmt, rule, shape):
     M, K = shape
     bs = 16 if fmt == "nvfp4" else 32
+    if K % bs:
+        pytest.skip("K not a multiple of the block")
     x = _adversarial_bf16(M, K, 3 * M + K, huge=3.0e38 if fmt != "nvfp4" else 3.0e6, bs=bs)
     g = 1.0
     gd = None

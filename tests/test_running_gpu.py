@@ -11,8 +11,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("layout", [mxq.SF_ROWMAJOR, mxq.SF_SWIZZLED])
-def test_running_max_sequence(layout):
-    M, K = 200, 1024
+@pytest.mark.parametrize("M,K", [(200, 1024), (3, 48)])
+def test_running_max_sequence(layout, M, K):
     state = [torch.tensor([0.75], dtype=torch.float32, device="cuda"), torch.empty(1, dtype=torch.float32, device="cuda")]
     ref_state = np.float32(0.75)
     for step, scale in enumerate([1.0, 3.0, 0.5, 8.0]):
