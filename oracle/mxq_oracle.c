@@ -28,6 +28,9 @@
  *   d = fl(dec(s) * g);  r = fl(1 / d);  v_i = fl(x_i * r);  q_i = RNE_E2M1_sat(v_i)
  * and a block whose d is 0 gets zero-magnitude codes that keep the sign of x.
  *
+ * The weight-only (W4A16) GEMM multiplies bf16 activations by dequantized MXFP4 / NVFP4 weights
+ * ("Qwen3.5-27B-NVFP4-RTN-weight-only": activations run bf16).
+ *
  * Parity status: every function here is pinned by the CPU test suite against library decoders
  * (ml_dtypes, torch), exact rational arithmetic or brute force, except the NVFP4 operation order
  * and the MXFP8 scale rule, which are readings (the pages do not fix them).
@@ -303,6 +306,49 @@ int orc_gemm(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Bq, const uin
     for (int64_t i = 0; i < nrows; i++) {
         int64_t m = rows ? rows[i] : i;
         for (int64_t k = 0; k < K; k++) arow[i * K + k] = dq_elem(Aq, Asf, m, k, K, fmt);
+    }
+    for (int64_t j = 0; j < ncols; j++) {
+        int64_t n = cols ? cols[j] : j;
+        for (int64_t k = 0; k < K; k++) brow[k] = dq_elem(Bq, Bsf, n, k, K, fmt);
+        for (int64_t i = 0; i < nrows; i++) {
+            double acc = 0.0, aacc = 0.0;
+            const double* a = arow + i * K;
+            for (int64_t k = 0; k < K; k++) {
+                double p = a[k] * brow[k];
+                acc += p;
+                aacc += fabs(p);
+            }
+            out[i * ncols + j] = alpha * acc;
+            if (abs_out) abs_out[i * ncols + j] = fabs(alpha) * aacc;
+        }
+    }
+    free(arow);
+    free(brow);
+    return 0;
+}
+
+/* Weight-only (W4A16) GEMM, the serving mode of "Qwen3.5-27B-NVFP4-RTN-weight-only" (first paragraph:
+ * the checkpoint's weights are NVFP4, activations run bf16) and the Marlin mode of
+ * "Qwen3.5-27B-MXFP4-QAD-W4A4-LR1e-5-s1000" ("Evaluation results": one artifact serves W4A4 and
+ * W4A16).  Out[i][j] = alpha * sum_k bf16(A[rows[i]][k]) * dq(B)[cols[j]][k] in fp64, alpha = gB for
+ * NVFP4 and 1 otherwise; abs_out likewise with |.|.  A is [M][K] bf16 bit patterns, B [N][K]
+ * quantized along K with row-major scales (MXFP4 or NVFP4).  Returns 0, or -1 when memory runs out. */
+int orc_gemm_w4a16(const uint16_t* A, const uint8_t* Bq, const uint8_t* Bsf, double gB, int64_t M, int64_t N,
+                   int64_t K, int fmt, const int64_t* rows, int64_t nrows, const int64_t* cols, int64_t ncols,
+                   double* out, double* abs_out) {
+    double alpha = fmt == ORC_NVFP4 ? gB : 1.0;
+    if (!rows) nrows = M;
+    if (!cols) ncols = N;
+    double* arow = (double*)malloc(sizeof(double) * (size_t)(nrows * K));
+    double* brow = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!arow || !brow) {
+        free(arow);
+        free(brow);
+        return -1;
+    }
+    for (int64_t i = 0; i < nrows; i++) {
+        int64_t m = rows ? rows[i] : i;
+        for (int64_t k = 0; k < K; k++) arow[i * K + k] = orc_bf16_value(A[m * K + k]);
     }
     for (int64_t j = 0; j < ncols; j++) {
         int64_t n = cols ? cols[j] : j;

@@ -50,6 +50,8 @@ def lib():
         L.orc_global_scale.argtypes, L.orc_global_scale.restype = [p, i64, p], f
         L.orc_gemm.argtypes = [p, p, p, p, d, d, i64, i64, i64, i32, p, i64, p, i64, p, p]
         L.orc_gemm.restype = i32
+        L.orc_gemm_w4a16.argtypes = [p, p, p, d, i64, i64, i64, i32, p, i64, p, i64, p, p]
+        L.orc_gemm_w4a16.restype = i32
         L.orc_f32_to_bf16.argtypes, L.orc_f32_to_bf16.restype = [f], ctypes.c_uint16
         L.orc_fake_quantize.argtypes, L.orc_fake_quantize.restype = [p, i64, i64, i32, i32, f, p], i32
         L.orc_quantize_running.argtypes, L.orc_quantize_running.restype = [p, i64, i64, f, p, p, p], i32
@@ -173,6 +175,25 @@ def gemm(Aq, Asf, Bq, Bsf, M, N, K, fmt, gA=1.0, gB=1.0, rows=None, cols=None):
     rc = lib().orc_gemm(_ptr(Aq), _ptr(Asf), _ptr(Bq), _ptr(Bsf), float(gA), float(gB), M, N, K, fmt,
                         None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
                         _ptr(out), _ptr(absout))
+    if rc != 0:
+        raise MemoryError("oracle gemm allocation failed")
+    return out, absout
+
+
+def gemm_w4a16(A, Bq, Bsf, M, N, K, fmt, gB=1.0, rows=None, cols=None):
+    """fp64 reference of Out = alpha * A @ dq(B)^T with A in bf16 (weight-only / W4A16 mode).
+    Returns (out, abs_sum), both [len(rows), len(cols)] float64."""
+    Ab = _bits(A)
+    Bq, Bsf = (np.ascontiguousarray(a, dtype=np.uint8) for a in (Bq, Bsf))
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
+    nr = M if r is None else r.size
+    nc = N if c is None else c.size
+    out = np.zeros((nr, nc), dtype=np.float64)
+    absout = np.zeros((nr, nc), dtype=np.float64)
+    rc = lib().orc_gemm_w4a16(_ptr(Ab), _ptr(Bq), _ptr(Bsf), float(gB), M, N, K, fmt,
+                              None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
+                              _ptr(out), _ptr(absout))
     if rc != 0:
         raise MemoryError("oracle gemm allocation failed")
     return out, absout
