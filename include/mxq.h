@@ -130,6 +130,26 @@ int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_
              const float* g_B, int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_out out_type, void* out,
              mxq_stream_t stream);
 
+/*
+ * Weight-only (W4A16) GEMM: out[M, N] = alpha * A dq(W)^T with bf16 activations A and MXFP4 or
+ * NVFP4 weights, alpha = g_W[0] for NVFP4 and 1 for MXFP4.  This is the weight-only serving mode:
+ * "Qwen3.5-27B-NVFP4-RTN-weight-only" (activations run bf16, no input_global_scale) and the
+ * Marlin mode of "Qwen3.5-27B-MXFP4-QAD-W4A4-LR1e-5-s1000" ("Evaluation results": one weight
+ * artifact serves W4A4 and W4A16).  W is dequantized to bf16 inside the kernel and multiplied on
+ * the tcgen05 tensor cores (bf16 x bf16, fp32 accumulation).
+ *   A        (device) [M, K] bf16, row-major.
+ *   W_q      (device) [N, K/2] packed E2M1 codes; W_sf (device) their SWIZZLED scales, the same
+ *            bytes mxq_gemm and mxq_linear read.
+ *   g_W      (device) fp32[1] NVFP4 global scale of W; ignored (may be NULL) for MXFP4.
+ *   out      (device) [M, N] bf16 (RNE) or fp32, row-major.
+ * Requires fmt MXQ_MXFP4 or MXQ_NVFP4 (else MXQ_ERR_UNSUPPORTED), M, N >= 1, K >= 64 with
+ * K % 64 == 0, 16-byte aligned pointers.  The dequantized weights are exact in bf16 for every
+ * scale the quantizer emits; scale codes it never emits (E8M0 0xFF, or 2^127 with code 6) are
+ * outside the contract.  Stream-ordered; allocates nothing.
+ */
+int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
+                   int64_t K, mxq_fmt fmt, mxq_out out_type, void* out, mxq_stream_t stream);
+
 /* Workspace bytes mxq_linear needs for M tokens of width K (quantized A plus swizzled scales). */
 size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt);
 

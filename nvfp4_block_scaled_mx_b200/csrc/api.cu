@@ -200,6 +200,17 @@ int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_
                        reinterpret_cast<cudaStream_t>(stream), false);
 }
 
+int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
+                   int64_t K, mxq_fmt fmt, mxq_out out_type, void* out, mxq_stream_t stream) {
+    if ((fmt != MXQ_MXFP4 && fmt != MXQ_NVFP4) || !valid_out(out_type)) return MXQ_ERR_UNSUPPORTED;
+    if (!A || !W_q || !W_sf || !out || (fmt == MXQ_NVFP4 && !g_W)) return MXQ_ERR_NULL;
+    int rc = validate_gemm_shape(M, N, K, fmt);
+    if (rc != MXQ_OK) return rc;
+    if (!aligned16(A) || !aligned16(W_q) || !aligned16(W_sf) || !aligned16(out)) return MXQ_ERR_ALIGN;
+    if ((rc = check_device()) != MXQ_OK) return rc;
+    return launch_w4a16(A, W_q, W_sf, g_W, M, N, K, fmt, out_type, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt) {
     if (!valid_fmt(fmt) || M < 1 || K < 1 || K % block_size(fmt) != 0) return 0;
     size_t qb = 0;

@@ -215,6 +215,23 @@ __device__ __forceinline__ uint32_t mma_idesc(uint32_t M, uint32_t N, uint32_t s
     return d;
 }
 
+// Instruction descriptor of a dense kind::f16 MMA with bf16 A and B (the same type on both
+// sides), fp32 accumulator, K-major operands: D format [4,6) = F32, A format [7,10) = BF16,
+// B format [10,13) = BF16, N>>3 [17,23), M>>4 [24,29).
+__device__ __forceinline__ uint32_t mma_idesc_bf16(uint32_t M, uint32_t N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulator, K = 16 per instruction.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // KIND 0: MXFP4 (kind::mxf4, E8M0 per 32 -> 2 scales per K=64 step)
 // KIND 1: NVFP4 (kind::mxf4nvf4, UE4M3 per 16 -> 4 scales per K=64 step)
 // KIND 2: MXFP8 (kind::mxf8f6f4, E8M0 per 32 -> 1 scale per K=32 step)
@@ -303,6 +320,23 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
 }
 
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)
+
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u8(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t saddr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+    return v;
+}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -423,6 +457,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ float e4m3_decode_pos(uint32_t code) {
     const uint32_t e = (code >> 3) & 0xFu, m = code & 7u;
     return e == 0 ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Two E2M1 codes (low nibble = first element) to an f16x2 (first element in the low half).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 a;\n\tcvt.u8.u32 a, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, a;\n\t}\n" : "=r"(r) : "r"(byte));
+    return r;
 }
 
 // 2^-e as fp32 for e in [-127, 127] (2^-127 is the subnormal 0x00400000).

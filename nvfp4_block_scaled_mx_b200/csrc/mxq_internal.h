@@ -47,6 +47,10 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
                 const float* g_B, int64_t M, int64_t N, int64_t K, int fmt, int out_type, void* out,
                 cudaStream_t stream, bool pdl_secondary);
 
+// Weight-only (W4A16) GEMM launch (arguments already validated).
+int launch_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
+                 int64_t K, int fmt, int out_type, void* out, cudaStream_t stream);
+
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace mxq

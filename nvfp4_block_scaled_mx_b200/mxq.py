@@ -34,6 +34,7 @@ SIGNATURES = {
     "mxq_swizzle_scales": (_I, [_P, _I64, _I64, _P, _P]),
     "mxq_global_scale": (_I, [_P, _I64, _P, _P, _P]),
     "mxq_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
+    "mxq_gemm_w4a16": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_linear_workspace_size": (_SZ, [_I64, _I64, _I]),
     "mxq_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _SZ, _P, _P]),
     "mxq_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
@@ -113,6 +114,10 @@ def mxq_global_scale(x, n, g_out, amax_out, stream):
 
 def mxq_gemm(A_q, A_sf, B_q, B_sf, g_A, g_B, M, N, K, fmt, out_type, out, stream):
     return lib().mxq_gemm(A_q, A_sf, B_q, B_sf, g_A, g_B, M, N, K, fmt, out_type, out, stream)
+
+
+def mxq_gemm_w4a16(A, W_q, W_sf, g_W, M, N, K, fmt, out_type, out, stream):
+    return lib().mxq_gemm_w4a16(A, W_q, W_sf, g_W, M, N, K, fmt, out_type, out, stream)
 
 
 def mxq_linear(x, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, workspace, ws_bytes, out, stream):
@@ -215,6 +220,18 @@ def gemm(A_q, A_sf, B_q, B_sf, M, N, K, fmt, out_dtype=torch.bfloat16, g_A=None,
         out = torch.empty((M, N), dtype=out_dtype, device=A_q.device)
     _check(mxq_gemm(_ptr(A_q), _ptr(A_sf), _ptr(B_q), _ptr(B_sf), _ptr(g_A), _ptr(g_B), M, N, K, f, ot, _ptr(out),
                     _stream(stream)), "mxq_gemm")
+    return out
+
+
+def gemm_w4a16(A, W_q, W_sf, N, fmt, g_W=None, out_dtype=torch.bfloat16, out=None, stream=None):
+    """Weight-only GEMM: out = A dq(W)^T with A [M, K] bf16 and W pre-quantized (swizzled scales)."""
+    f = _fmt(fmt)
+    M, K = A.shape
+    ot = OUT_FP32 if out_dtype == torch.float32 else OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    _check(mxq_gemm_w4a16(_ptr(A), _ptr(W_q), _ptr(W_sf), _ptr(g_W), M, N, K, f, ot, _ptr(out), _stream(stream)),
+           "mxq_gemm_w4a16")
     return out
 
 
