@@ -303,8 +303,9 @@ def run_mxq(args, world, rank, local):
 
 
 def other_workloads(stream, bf16_tflops):
-    """mxq_linear on the remaining problems (decode, NVFP4 down-proj, MXFP8 attention, lm_head):
-    device-resident inputs, CUDA events, informational (the headline is the prefill problem)."""
+    """mxq_linear on the remaining problems (decode, NVFP4 down-proj, MXFP8 attention, lm_head, N = 96)
+    and the weight-only GEMM on the prefill and decode shapes: device-resident inputs, CUDA events,
+    informational (the headline is the prefill problem)."""
     from nvfp4_block_scaled_mx_b200 import mxq
     res = {}
     for name in ["decode", "down_nvfp4", "attn_mxfp8", "lm_head", "in_proj_ba"]:
@@ -342,6 +343,27 @@ def other_workloads(stream, bf16_tflops):
             del q, sf, flush
         res[name] = r
         del A, W_q, W_sf, ws, out
+        torch.cuda.empty_cache()
+    # weight-only (W4A16): bf16 activations times the same MXFP4 weights, on the prefill gate+up and
+    # decode shapes; tensor-bound against the measured bf16 peak at prefill, weight-stream-bound at decode
+    for name in ["prefill_gate_up", "decode"]:
+        cfg = synth.CONFIGS[name]
+        M, N, K = cfg["M"], cfg["N"], cfg["K"]
+        A, W = synth.make_inputs(name, device="cuda")
+        W_q, W_sf = mxq.quantize(W, "mxfp4", "even")
+        del W
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        f = lambda: mxq.gemm_w4a16(A, W_q, W_sf, N, "mxfp4", out=out, stream=stream)
+        for _ in range(3):
+            f()
+        t = time_loop(f, 200 if M * N < 1e8 else 10, stream)
+        r = {"M": M, "N": N, "K": K, "fmt": "mxfp4 weights, bf16 activations", "ms": round(t * 1e3, 4),
+             "tflops": round(2.0 * M * N * K / t / 1e12, 1),
+             "frac_of_measured_bf16": round(2.0 * M * N * K / t / 1e12 / bf16_tflops, 4)}
+        if name == "decode":
+            r["weight_gbs"] = round((W_q.numel() + W_sf.numel()) / t / 1e9, 1)
+        res["w4a16_" + name] = r
+        del A, W_q, W_sf, out
         torch.cuda.empty_cache()
     return res
 

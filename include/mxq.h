@@ -144,8 +144,8 @@ int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_
  *   out      (device) [M, N] bf16 (RNE) or fp32, row-major.
  * Requires fmt MXQ_MXFP4 or MXQ_NVFP4 (else MXQ_ERR_UNSUPPORTED), M, N >= 1, K >= 64 with
  * K % 64 == 0, 16-byte aligned pointers.  The dequantized weights are exact in bf16 for every
- * scale the quantizer emits; scale codes it never emits (E8M0 0xFF, or 2^127 with code 6) are
- * outside the contract.  Stream-ordered; allocates nothing.
+ * scale the EVEN-rule weight quantizer emits (E8M0 codes up to 252, E4M3 codes up to 0x7E); larger
+ * E8M0 codes can overflow and are outside the contract.  Stream-ordered; allocates nothing.
  */
 int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
                    int64_t K, mxq_fmt fmt, mxq_out out_type, void* out, mxq_stream_t stream);

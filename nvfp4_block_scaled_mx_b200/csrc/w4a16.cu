@@ -69,8 +69,10 @@ __device__ __forceinline__ float pow2f(int e) {
     return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
 }
 
-// 8 E2M1 codes (one 32-bit word, first element in the low nibble) times `scale`, as 4 bf16x2 words.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, float scale) {
+// 8 E2M1 codes (one 32-bit word, first element in the low nibble) times `scale`, as 4 bf16x2 words,
+// through the conversion pipe (cvt e2m1x2 -> f16x2, fp32 multiply, cvt -> bf16x2).  Exact for every
+// scale; used where the bf16 product could leave the normal range.
+__device__ __forceinline__ uint4 dequant8_cvt(uint32_t w, float scale) {
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -79,6 +81,33 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, float scale) {
         const __nv_bfloat162 b =
             __floats2bfloat162_rn(__fmul_rn(__low2float(hh), scale), __fmul_rn(__high2float(hh), scale));
         o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The same on the integer and FMA pipes: the bf16 bit patterns of the E2M1 magnitudes 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6 come from byte-permute lookups (high and low byte tables, 3-bit selectors), the
+// sign bits are moved to bit 15, and a bf16x2 multiply applies the scale s2 = (s, s).  Exact when
+// every product is a normal bf16: the scale lies in [2^-125, 2^125] (MXFP4) or is an E4M3 value
+// (NVFP4; products in [2^-10, 2688]).
+__device__ __forceinline__ uint4 dequant8_prmt(uint32_t w, uint32_t s2) {
+    constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u;  // high bytes of magnitudes 0-3, 4-7
+    constexpr uint32_t kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;  // low bytes
+    const uint32_t m0 = w & 0x7777u, m1 = (w >> 16) & 0x7777u;   // magnitudes as byte selectors
+    uint32_t hi0 = __byte_perm(kHiLo, kHiHi, m0), lo0 = __byte_perm(kLoLo, kLoHi, m0);
+    uint32_t hi1 = __byte_perm(kHiLo, kHiHi, m1), lo1 = __byte_perm(kLoLo, kLoHi, m1);
+    // sign of code i (bit 4i + 3) to bit 7 of byte i: even codes come from sg << 4, odd codes from sg
+    const uint32_t sg = w & 0x88888888u, sh = sg << 4;
+    hi0 |= __byte_perm(sg, sh, 0x1504) & 0x80808080u;
+    hi1 |= __byte_perm(sg, sh, 0x3726) & 0x80808080u;
+    const uint32_t p[4] = {__byte_perm(lo0, hi0, 0x5140), __byte_perm(lo0, hi0, 0x7362), __byte_perm(lo1, hi1, 0x5140),
+                           __byte_perm(lo1, hi1, 0x7362)};
+    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]), sc);
+        o[i] = *reinterpret_cast<const uint32_t*>(&v);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -244,20 +273,39 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                 for (int i = 0; i < ITEMS; ++i) {
                     const int id = t + 128 * i;
                     const int row = id % BN, half = id / BN;
-                    float s0, s1;
-                    if constexpr (FMT == MXQ_NVFP4) {
-                        const uint32_t c0 = sc[i] & 0xFFu, c1 = sc[i] >> 8;
-                        s0 = e4m3_decode_pos(c0 & 0x7Fu) * ((c0 & 0x80u) ? -1.0f : 1.0f);
-                        s1 = e4m3_decode_pos(c1 & 0x7Fu) * ((c1 & 0x80u) ? -1.0f : 1.0f);
-                    } else {
-                        s0 = s1 = pow2f(static_cast<int>(sc[i]) - 127);
-                    }
                     const uint32_t rbase = b_s + row * 128;
                     const uint32_t sw = static_cast<uint32_t>(row & 7);
-                    st_shared_v4(rbase + (((4 * half + 0) ^ sw) << 4), dequant8(codes[i].x, s0));
-                    st_shared_v4(rbase + (((4 * half + 1) ^ sw) << 4), dequant8(codes[i].y, s0));
-                    st_shared_v4(rbase + (((4 * half + 2) ^ sw) << 4), dequant8(codes[i].z, s1));
-                    st_shared_v4(rbase + (((4 * half + 3) ^ sw) << 4), dequant8(codes[i].w, s1));
+                    uint4 o0, o1, o2, o3;
+                    if constexpr (FMT == MXQ_NVFP4) {
+                        // E4M3 block scales (exact in bf16); the first 16 elements take s0, the rest s1
+                        const uint32_t c0 = sc[i] & 0xFFu, c1 = sc[i] >> 8;
+                        const __nv_bfloat16 b0 = __float2bfloat16_rn(e4m3_decode_pos(c0 & 0x7Fu) * ((c0 & 0x80u) ? -1.0f : 1.0f));
+                        const __nv_bfloat16 b1 = __float2bfloat16_rn(e4m3_decode_pos(c1 & 0x7Fu) * ((c1 & 0x80u) ? -1.0f : 1.0f));
+                        const uint32_t u0 = *reinterpret_cast<const uint16_t*>(&b0), u1 = *reinterpret_cast<const uint16_t*>(&b1);
+                        o0 = dequant8_prmt(codes[i].x, u0 * 0x10001u);
+                        o1 = dequant8_prmt(codes[i].y, u0 * 0x10001u);
+                        o2 = dequant8_prmt(codes[i].z, u1 * 0x10001u);
+                        o3 = dequant8_prmt(codes[i].w, u1 * 0x10001u);
+                    } else {
+                        const int e = static_cast<int>(sc[i]) - 127;
+                        if (e >= -125 && e <= 125) {
+                            const uint32_t s2 = (static_cast<uint32_t>(e + 127) << 7) * 0x10001u;  // bf16 2^e, twice
+                            o0 = dequant8_prmt(codes[i].x, s2);
+                            o1 = dequant8_prmt(codes[i].y, s2);
+                            o2 = dequant8_prmt(codes[i].z, s2);
+                            o3 = dequant8_prmt(codes[i].w, s2);
+                        } else {
+                            const float s = pow2f(e);
+                            o0 = dequant8_cvt(codes[i].x, s);
+                            o1 = dequant8_cvt(codes[i].y, s);
+                            o2 = dequant8_cvt(codes[i].z, s);
+                            o3 = dequant8_cvt(codes[i].w, s);
+                        }
+                    }
+                    st_shared_v4(rbase + (((4 * half + 0) ^ sw) << 4), o0);
+                    st_shared_v4(rbase + (((4 * half + 1) ^ sw) << 4), o1);
+                    st_shared_v4(rbase + (((4 * half + 2) ^ sw) << 4), o2);
+                    st_shared_v4(rbase + (((4 * half + 3) ^ sw) << 4), o3);
                 }
                 fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor cores
                 __syncwarp();

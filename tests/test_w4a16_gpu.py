@@ -87,6 +87,21 @@ def test_w4a16_scale_placement(fmt, M):
     check_fp32(gpu, ref, abs_sum, "%s scales" % fmt)
 
 
+@pytest.mark.parametrize("codes,a_scale", [((0, 1, 2, 3, 4), 2.0 ** 100), ((248, 249, 250, 251, 252), 2.0 ** -100)])
+def test_w4a16_extreme_mx_scales(codes, a_scale):
+    """E8M0 scales at the ends of the range: 2^-127 and 2^-126 dequantize through the exact fp32
+    path (bf16 subnormal products), 2^-125 ... 2^125 through the byte-permute path.  Activations
+    are scaled so that the products and sums stay normal fp32 numbers."""
+    M, N, K = 130, 96, 256
+    rng = np.random.default_rng(codes[0])
+    A = (synth.random_bf16((M, K), 61).float() * a_scale).to(torch.bfloat16)
+    Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    Wsf = rng.choice(np.array(codes, np.uint8), (N, K // 32)).astype(np.uint8)
+    ref, abs_sum = oracle.gemm_w4a16(A, Wq, Wsf, M, N, K, oracle.MXFP4)
+    gpu = _gpu_w4a16(A, (Wq, Wsf, 1.0), N, "mxfp4", torch.float32)
+    check_fp32(gpu, ref, abs_sum, "extreme scales %s" % (codes,))
+
+
 def test_w4a16_rejects_mxfp8_and_bad_shapes():
     A = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
     Wq = torch.zeros(8, 32, dtype=torch.uint8, device="cuda")
