@@ -93,13 +93,13 @@ __device__ __forceinline__ uint4 dequant8_cvt(uint32_t w, float scale) {
 __device__ __forceinline__ uint4 dequant8_prmt(uint32_t w, uint32_t s2) {
     constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u;  // high bytes of magnitudes 0-3, 4-7
     constexpr uint32_t kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;  // low bytes
-    const uint32_t m0 = w & 0x7777u, m1 = (w >> 16) & 0x7777u;   // magnitudes as byte selectors
+    const uint32_t m0 = w & 0x77777777u, m1 = m0 >> 16;           // magnitudes as byte selectors (low 16 bits)
     uint32_t hi0 = __byte_perm(kHiLo, kHiHi, m0), lo0 = __byte_perm(kLoLo, kLoHi, m0);
     uint32_t hi1 = __byte_perm(kHiLo, kHiHi, m1), lo1 = __byte_perm(kLoLo, kLoHi, m1);
-    // sign of code i (bit 4i + 3) to bit 7 of byte i: even codes come from sg << 4, odd codes from sg
-    const uint32_t sg = w & 0x88888888u, sh = sg << 4;
-    hi0 |= __byte_perm(sg, sh, 0x1504) & 0x80808080u;
-    hi1 |= __byte_perm(sg, sh, 0x3726) & 0x80808080u;
+    // the sign of code i (bit 4i + 3) is bit 7 of byte i / 2 of w << 4 (even i) or of w (odd i)
+    const uint32_t sh = w << 4;
+    hi0 |= __byte_perm(sh, w, 0x5140) & 0x80808080u;
+    hi1 |= __byte_perm(sh, w, 0x7362) & 0x80808080u;
     const uint32_t p[4] = {__byte_perm(lo0, hi0, 0x5140), __byte_perm(lo0, hi0, 0x7362), __byte_perm(lo1, hi1, 0x5140),
                            __byte_perm(lo1, hi1, 0x7362)};
     const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
@@ -110,6 +110,19 @@ __device__ __forceinline__ uint4 dequant8_prmt(uint32_t w, uint32_t s2) {
         o[i] = *reinterpret_cast<const uint32_t*>(&v);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// True if the E8M0 codes in the low `n` bytes of `codes` all lie in [2, 252] (scales 2^-125 ..
+// 2^125), where dequant8_prmt is exact.
+__device__ __forceinline__ bool mx_scales_in_range(uint32_t codes, int n) {
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (i < n) {
+            const uint32_t b = (codes >> (8 * i)) & 0xFFu;
+            ok = ok && b >= 2u && b <= 252u;
+        }
+    return ok;
 }
 
 template <int FMT, int BMT, int BN, bool OUT_F32>
@@ -269,6 +282,14 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage's W bytes
                 const uint32_t b_s = smem_u32(smem + C::OFF_B + buf * C::B_BYTES);
+                // MXFP4: the byte-permute path unless some scale of the warp's items leaves 2^-125 .. 2^125
+                bool fast = true;
+                if constexpr (FMT != MXQ_NVFP4) {
+                    bool mine = true;
+#pragma unroll
+                    for (int i = 0; i < ITEMS; ++i) mine = mine && mx_scales_in_range(sc[i], 1);
+                    fast = __all_sync(0xFFFFFFFFu, mine);
+                }
 #pragma unroll
                 for (int i = 0; i < ITEMS; ++i) {
                     const int id = t + 128 * i;
@@ -286,21 +307,18 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                         o1 = dequant8_prmt(codes[i].y, u0 * 0x10001u);
                         o2 = dequant8_prmt(codes[i].z, u1 * 0x10001u);
                         o3 = dequant8_prmt(codes[i].w, u1 * 0x10001u);
+                    } else if (fast) {
+                        const uint32_t s2 = (sc[i] << 7) * 0x10001u;  // bf16 2^(code - 127), twice
+                        o0 = dequant8_prmt(codes[i].x, s2);
+                        o1 = dequant8_prmt(codes[i].y, s2);
+                        o2 = dequant8_prmt(codes[i].z, s2);
+                        o3 = dequant8_prmt(codes[i].w, s2);
                     } else {
-                        const int e = static_cast<int>(sc[i]) - 127;
-                        if (e >= -125 && e <= 125) {
-                            const uint32_t s2 = (static_cast<uint32_t>(e + 127) << 7) * 0x10001u;  // bf16 2^e, twice
-                            o0 = dequant8_prmt(codes[i].x, s2);
-                            o1 = dequant8_prmt(codes[i].y, s2);
-                            o2 = dequant8_prmt(codes[i].z, s2);
-                            o3 = dequant8_prmt(codes[i].w, s2);
-                        } else {
-                            const float s = pow2f(e);
-                            o0 = dequant8_cvt(codes[i].x, s);
-                            o1 = dequant8_cvt(codes[i].y, s);
-                            o2 = dequant8_cvt(codes[i].z, s);
-                            o3 = dequant8_cvt(codes[i].w, s);
-                        }
+                        const float s = pow2f(static_cast<int>(sc[i]) - 127);
+                        o0 = dequant8_cvt(codes[i].x, s);
+                        o1 = dequant8_cvt(codes[i].y, s);
+                        o2 = dequant8_cvt(codes[i].z, s);
+                        o3 = dequant8_cvt(codes[i].w, s);
                     }
                     st_shared_v4(rbase + (((4 * half + 0) ^ sw) << 4), o0);
                     st_shared_v4(rbase + (((4 * half + 1) ^ sw) << 4), o1);
@@ -397,6 +415,402 @@ __global__ void __launch_bounds__(kW16Threads, 1)
     }
 }
 
+// ------------------------------------------------------------------ weights dequantized into TMEM
+//
+// For few tokens (M <= 128) the weights dominate the traffic.  Here Out^T tile = W tile [128 weight
+// rows] x A tile^T [NT tokens]: the MMA's A operand is the dequantized weight tile, which the
+// dequant warps write straight into TMEM (tcgen05.st: a thread's TMEM lane is its weight row), and
+// its B operand is the bf16 activation tile in shared memory.  K advances 256 per stage, so each
+// weight row contributes a full 128-byte line per stage (the 128 rows arrive as one 16 KB TMA box
+// with a 128-byte swizzle).
+//   warp 0       TMA producer: 4 activation boxes (NT tokens x 64 K, 128B-swizzled), 128 rows of
+//                packed codes (128 bytes each), their scale tiles
+//   warp 1       TMEM owner; MMA issuer (A from TMEM, B from shared memory), 16 MMAs per stage
+//   warps 2-9    dequantization into TMEM slots of 128 columns: two warps per sub-partition, each
+//                converting 128 of the stage's 256 K elements of its 32 rows
+//   warps 10-17  epilogue: a lane owns one weight row (output column), so a warp's store for one
+//                token covers 32 consecutive output columns
+// SPLIT: a cluster of k_split CTAs shares one tile, each CTA a contiguous range of K stages, and
+// the partials are reduced through distributed shared memory in the leader.  Otherwise the grid is
+// persistent over tiles (tokens fastest) with two accumulators when TMEM has room.
+
+constexpr int kWtDeqWarps = 8;  // 16 (the epilogue warps too) when every CTA owns one tile
+constexpr int kWtEpiWarps = 8;
+constexpr int kWtThreads = (2 + kWtDeqWarps + kWtEpiWarps) * 32;
+constexpr int kWtK = 256;  // K elements per stage
+
+template <int FMT, int NT, int STAGES, int AS, bool SPLIT>
+struct W16TCfg {
+    static constexpr int BS = (FMT == MXQ_NVFP4) ? 16 : 32;
+    static constexpr int SF_ATOMS = kWtK / BS / 4;           // 512-byte scale tiles per stage (2 or 4)
+    static constexpr int ACT_SUB = NT * 128;                 // one activation box: NT rows x 128 bytes
+    static constexpr int ACT_BYTES = 4 * ACT_SUB;
+    static constexpr int W_BYTES = 128 * 128;
+    static constexpr int SF_BYTES = SF_ATOMS * 512;
+    static constexpr int ACC = (!SPLIT && 2 * NT + AS * 128 <= 512) ? 2 : 1;
+    static constexpr int A_TMEM = ACC * NT;  // first column of the weight slots
+    static constexpr int COLS_USED = A_TMEM + AS * 128;
+    static constexpr uint32_t TMEM_COLS = COLS_USED <= 256 ? 256u : 512u;
+    static constexpr int OFF_ACT = 0;
+    static constexpr int OFF_W = OFF_ACT + STAGES * ACT_BYTES;
+    static constexpr int OFF_SF = OFF_W + STAGES * W_BYTES;
+    static constexpr int OFF_BAR = OFF_SF + STAGES * SF_BYTES;
+    static constexpr int N_BARS = 2 * STAGES + 2 * AS + 2 * ACC;
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
+    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N");
+    static_assert(COLS_USED <= 512, "TMEM budget");
+    static_assert(ACT_SUB % 1024 == 0, "128B-swizzled activation boxes stay 1024-byte aligned");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct W16TArgs {
+    const float* g_w;
+    void* out;
+    int M, N, K;
+    int sf_col_tiles;
+    int t_tiles, w_tiles, k_stages;
+    uint32_t k_split;
+    uint32_t act_box_bytes;
+    int* status;
+};
+
+template <int FMT, int NT, int STAGES, int AS, bool SPLIT, int DQW, bool OUT_F32>
+__global__ void __launch_bounds__(kWtThreads, 1)
+    w4a16_tmem_kernel(const __grid_constant__ CUtensorMap tma_act, const __grid_constant__ CUtensorMap tma_w,
+                      const __grid_constant__ CUtensorMap tma_sf, const W16TArgs p) {
+    using C = W16TCfg<FMT, NT, STAGES, AS, SPLIT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // activations, codes, scales landed
+    uint64_t* empty = full + STAGES;                                   // MMAs read activations, dequant read codes
+    uint64_t* aready = empty + STAGES;                                 // weight slot written
+    uint64_t* aempty = aready + AS;                                    // MMAs done with the weight slot
+    uint64_t* accf = aempty + AS;                                      // accumulator ready
+    uint64_t* acce = accf + C::ACC;                                    // accumulator drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t split = 0, splits = 1;
+    if constexpr (SPLIT) {
+        split = cluster_ctarank();
+        splits = p.k_split;
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_act);
+        prefetch_tmap(&tma_w);
+        prefetch_tmap(&tma_sf);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + DQW);
+        }
+        for (int a = 0; a < AS; ++a) {
+            mbar_init(&aready[a], DQW);
+            mbar_init(&aempty[a], 1);
+        }
+        for (int b = 0; b < C::ACC; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], kWtEpiWarps);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // tiles: tokens fastest; a SPLIT cluster takes one tile and a contiguous range of K stages
+    const int num_tiles = p.t_tiles * p.w_tiles;
+    const int first = SPLIT ? static_cast<int>(blockIdx.x / splits) : static_cast<int>(blockIdx.x);
+    const int step = SPLIT ? num_tiles : static_cast<int>(gridDim.x);
+    const int per = (p.k_stages + static_cast<int>(splits) - 1) / static_cast<int>(splits);
+    const int k0 = static_cast<int>(split) * per;
+    const int k1 = min(p.k_stages, k0 + per);
+
+    if (warp == 0) {
+        const uint64_t pol_act = policy_evict_last();  // activation tiles are reused by every weight tile
+        const uint64_t pol_w = policy_evict_first();   // weights stream
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = first; tile < num_tiles && ok; tile += step) {
+            const int tt = tile % p.t_tiles, wt = tile / p.t_tiles;
+            for (int ks = k0; ks < k1; ++ks) {
+                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 51)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[stage], 4 * p.act_box_bytes + C::W_BYTES + C::SF_BYTES);
+                    uint8_t* act = smem + C::OFF_ACT + stage * C::ACT_BYTES;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b)
+                        tma_load_2d(&tma_act, &full[stage], act + b * C::ACT_SUB, ks * kWtK + b * 64, tt * NT, pol_act);
+                    tma_load_2d(&tma_w, &full[stage], smem + C::OFF_W + stage * C::W_BYTES, ks * (kWtK / 2), wt * 128,
+                                pol_w);
+                    // the stage's SF_ATOMS consecutive 512-byte scale tiles of these 128 rows
+                    tma_load_2d(&tma_sf, &full[stage], smem + C::OFF_SF + stage * C::SF_BYTES, 0,
+                                (wt * p.sf_col_tiles + ks * C::SF_ATOMS) * 2, pol_w);
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        const uint32_t idesc = mma_idesc_bf16(128, NT);
+        int stage = 0, slot = 0, acc = 0;
+        uint32_t phase = 0, sphase = 0, acc_phase = 0;
+        bool ok = true;
+        for (int tile = first; tile < num_tiles && ok; tile += step) {
+            if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1u, p.status, 52)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NT);
+            for (int ks = k0; ks < k1; ++ks) {
+                if (!mbar_wait_warp(&full[stage], phase, p.status, 53) ||
+                    !mbar_wait_warp(&aready[slot], sphase, p.status, 54)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t act_s = smem_u32(smem + C::OFF_ACT + stage * C::ACT_BYTES);
+                const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_TMEM + slot * 128);
+                if (elect_one()) {
+#pragma unroll
+                    for (int j = 0; j < kWtK / 16; ++j)
+                        mma_bf16_ts(d_tmem, a_tmem + j * 8,
+                                    smem_desc(act_s + (j >> 2) * C::ACT_SUB + (j & 3) * 32, 16, 1024, kLayoutSwizzle128B),
+                                    idesc, (ks > k0 || j > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    tc_commit(&aempty[slot]);
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++slot == AS) {
+                    slot = 0;
+                    sphase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (elect_one()) tc_commit(&accf[acc]);
+            __syncwarp();
+            if (++acc == C::ACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    } else if (warp < 2 + DQW) {
+        // dequantization: this thread's weight row of the tile is its TMEM lane; warp group kq
+        // converts K elements [KE * kq, + KE) of the stage (KE / 2 bytes of codes, NBLK scale blocks)
+        // into TMEM columns [KE / 2 * kq, + KE / 2) of the slot, 64 elements at a time
+        constexpr int KE = 4 * kWtK / DQW;   // 128 or 64
+        constexpr int NCH = KE / 32;         // 16-byte code pieces per thread
+        constexpr int NBLK = KE / C::BS;     // scale blocks per thread
+        constexpr int NSW = (NBLK + 3) / 4;  // 32-bit scale words per thread
+        const int r = 32 * (warp & 3) + lane;
+        const int kq = (warp - 2) >> 2;
+        const int blk0 = NBLK * kq;  // the warp's first scale block in the stage
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const uint32_t sw = static_cast<uint32_t>(r & 7);  // 128-byte swizzle of the code rows
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
+        bool ok = true;
+        for (int tile = first; tile < num_tiles && ok; tile += step) {
+            for (int ks = k0; ks < k1; ++ks) {
+                if (!mbar_wait_warp(&full[stage], phase, p.status, 55)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t w_row = smem_u32(smem + C::OFF_W + stage * C::W_BYTES) + r * 128;
+                uint4 c[NCH];
+#pragma unroll
+                for (int q = 0; q < NCH; ++q) c[q] = ld_shared_v4(w_row + (((NCH * kq + q) ^ sw) << 4));
+                // a 512-byte scale tile holds 4 consecutive blocks of each of the 128 rows
+                const uint32_t sf_row = smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES) + (r & 31) * 16 + (r >> 5) * 4;
+                uint32_t sc[NSW];
+#pragma unroll
+                for (int i = 0; i < NSW; ++i)
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc[i]) : "r"(sf_row + ((blk0 >> 2) + i) * 512));
+                if constexpr (NBLK < 4) sc[0] >>= 8 * (blk0 & 3);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage's codes and scales
+                if (!mbar_wait_warp(&aempty[slot], sphase ^ 1u, p.status, 56)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t t_col =
+                    tmem_base + lane_addr + static_cast<uint32_t>(C::A_TMEM + slot * 128 + kq * (KE / 2));
+                // MXFP4: the byte-permute path unless some scale of the warp leaves 2^-125 .. 2^125
+                const bool fast = (FMT == MXQ_NVFP4) || __all_sync(0xFFFFFFFFu, mx_scales_in_range(sc[0], NBLK));
+                if (fast) {
+                    uint32_t s2[NBLK];  // block scales as bf16x2 (s, s)
+#pragma unroll
+                    for (int b = 0; b < NBLK; ++b) {
+                        const uint32_t code = (sc[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+                        if constexpr (FMT == MXQ_NVFP4) {
+                            const __nv_bfloat16 h =
+                                __float2bfloat16_rn(e4m3_decode_pos(code & 0x7Fu) * ((code & 0x80u) ? -1.0f : 1.0f));
+                            s2[b] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) * 0x10001u;
+                        } else {
+                            s2[b] = (code << 7) * 0x10001u;  // bf16 2^(code - 127)
+                        }
+                    }
+#pragma unroll
+                    for (int hq = 0; hq < KE / 64; ++hq) {  // 64 elements (two 16-byte code pieces) at a time
+                        uint32_t v[32];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int wi = 8 * hq + j;  // word index in this warp's KE elements
+                            const uint4 cc = c[wi >> 2];
+                            const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
+                            const uint4 o = dequant8_prmt(word, s2[wi * 8 / C::BS]);
+                            v[4 * j + 0] = o.x;
+                            v[4 * j + 1] = o.y;
+                            v[4 * j + 2] = o.z;
+                            v[4 * j + 3] = o.w;
+                        }
+                        tmem_st_cols<32>(t_col + hq * 32, v);
+                    }
+                } else {
+#pragma unroll
+                    for (int hq = 0; hq < KE / 64; ++hq) {
+                        uint32_t v[32];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int wi = 8 * hq + j;
+                            const uint4 cc = c[wi >> 2];
+                            const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
+                            const uint32_t code = (sc[0] >> (8 * (wi >> 2))) & 0xFFu;
+                            const uint4 o = dequant8_cvt(word, pow2f(static_cast<int>(code) - 127));
+                            v[4 * j + 0] = o.x;
+                            v[4 * j + 1] = o.y;
+                            v[4 * j + 2] = o.z;
+                            v[4 * j + 3] = o.w;
+                        }
+                        tmem_st_cols<32>(t_col + hq * 32, v);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aready[slot]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++slot == AS) {
+                    slot = 0;
+                    sphase ^= 1u;
+                }
+            }
+        }
+    }
+
+    // epilogue: warp e drains TMEM sub-partition (warp % 4), i.e. weight rows 32 * sub .. + 31, and
+    // token columns [half * NT / 2, + NT / 2) of the tile
+    constexpr int HC = NT / 2;
+    const bool epi = warp >= 2 + kWtDeqWarps;
+    const int sub = warp & 3;
+    const int half = (warp - 2 - kWtDeqWarps) >> 2;
+    const float alpha = (FMT == MXQ_NVFP4) ? *p.g_w : 1.0f;
+    auto store = [&](int tt, int wt, int j, float val) {
+        const int tok = tt * NT + half * HC + j, n = wt * 128 + sub * 32 + lane;
+        if (tok < p.M && n < p.N) {
+            const float y = __fmul_rn(val, alpha);
+            if constexpr (OUT_F32)
+                static_cast<float*>(p.out)[static_cast<int64_t>(tok) * p.N + n] = y;
+            else
+                static_cast<__nv_bfloat16*>(p.out)[static_cast<int64_t>(tok) * p.N + n] = __float2bfloat16_rn(y);
+        }
+    };
+    if constexpr (!SPLIT) {
+        if (epi) {
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int tile = first; tile < num_tiles; tile += step) {
+                const int tt = tile % p.t_tiles, wt = tile / p.t_tiles;
+                if (!mbar_wait(&accf[acc], acc_phase, p.status, 57)) break;
+                tc_fence_after();
+                const uint32_t t_row =
+                    tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * NT + half * HC);
+#pragma unroll 1
+                for (int c = 0; c < HC; c += 16) {
+                    uint32_t rr[16];
+                    tmem_ld_32x32b_x16(t_row + c, rr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) store(tt, wt, c + j, __uint_as_float(rr[j]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[acc]);
+                if (++acc == C::ACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    } else {
+        // every CTA's epilogue warps take their partial tile into registers
+        float part[HC];
+        if (epi) {
+            const bool ok = mbar_wait(&accf[0], 0, p.status, 58);
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(half * HC);
+#pragma unroll
+            for (int c = 0; c < HC; c += 16) {
+                uint32_t rr[16];
+                tmem_ld_32x32b_x16(t_row + c, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) part[c + j] = ok ? __uint_as_float(rr[j]) : 0.0f;
+            }
+            tc_fence_before();
+        }
+        // 1: every CTA's MMAs are done, so the leader's operand ring is free for the partials
+        __syncthreads();
+        cluster_sync();
+        float* red = reinterpret_cast<float*>(smem);  // leader: [splits-1][128 rows][NT] fp32
+        const int row = sub * 32 + lane;
+        if (epi && split != 0) {
+            const uint32_t dst = mapa_shared(smem_u32(red + ((split - 1) * 128 + row) * NT + half * HC), 0);
+#pragma unroll
+            for (int v4 = 0; v4 < HC / 4; ++v4)
+                asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + v4 * 16), "f"(part[4 * v4]),
+                             "f"(part[4 * v4 + 1]), "f"(part[4 * v4 + 2]), "f"(part[4 * v4 + 3])
+                             : "memory");
+        }
+        // 2: all partials sit in the leader's shared memory
+        cluster_sync();
+        if (epi && split == 0) {
+            const int tt = first % p.t_tiles, wt = first / p.t_tiles;
+            for (uint32_t sp = 1; sp < splits; ++sp) {
+                const float* src = red + ((sp - 1) * 128 + row) * NT + half * HC;
+#pragma unroll
+                for (int j = 0; j < HC; ++j) part[j] = __fadd_rn(part[j], src[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < HC; ++j) store(tt, wt, j, part[j]);
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // bf16 A [M][K]: boxes of 64 elements (128 bytes) x box_rows, 128B swizzle.
 bool make_a16_map(CUtensorMap* m, const void* A, int64_t M, int64_t K, uint32_t box_rows) {
     auto enc = encode_fn();
@@ -431,6 +845,33 @@ bool make_w_sf_map(CUtensorMap* m, const void* sf, int64_t rows, int64_t kblocks
     cuuint64_t dims[2] = {256, half_rows};
     cuuint64_t strides[1] = {256};
     cuuint32_t box[2] = {256, 2};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sf), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// packed FP4 W [N][K/2]: boxes of 128 bytes (256 elements) x 128 rows, 128B swizzle.
+bool make_w4_wide_map(CUtensorMap* m, const void* W, int64_t N, int64_t K) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(W), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Swizzled W scales as rows of 256 bytes; a box is `tiles` consecutive 512-byte tiles of a row group.
+bool make_w_sf_tiles_map(CUtensorMap* m, const void* sf, int64_t rows, int64_t kblocks, uint32_t tiles) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const uint64_t half_rows = static_cast<uint64_t>(swizzled_sf_bytes(rows, kblocks) / 256);
+    cuuint64_t dims[2] = {256, half_rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, 2 * tiles};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sf), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -473,13 +914,90 @@ int run_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w,
     return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+template <int FMT, int NT, int STAGES, int AS, bool SPLIT, int DQW, bool F32>
+int run_w16t(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w, int64_t M, int64_t N, int64_t K,
+             void* out, cudaStream_t stream, int splits) {
+    using C = W16TCfg<FMT, NT, STAGES, AS, SPLIT>;
+    auto kern = w4a16_tmem_kernel<FMT, NT, STAGES, AS, SPLIT, DQW, F32>;
+    const uint32_t act_rows = static_cast<uint32_t>(M >= NT ? NT : ceil_div(M, 8) * 8);
+    CUtensorMap ta, tw, tsf;
+    if (!make_a16_map(&ta, A, M, K, act_rows) || !make_w4_wide_map(&tw, Wq, N, K) ||
+        !make_w_sf_tiles_map(&tsf, Wsf, N, K / C::BS, C::SF_ATOMS))
+        return MXQ_ERR_CUDA;
+    W16TArgs args = {};
+    args.g_w = g_w;
+    args.out = out;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(N);
+    args.K = static_cast<int>(K);
+    args.sf_col_tiles = static_cast<int>(ceil_div(K / C::BS, 4));
+    args.t_tiles = static_cast<int>(ceil_div(M, NT));
+    args.w_tiles = static_cast<int>(ceil_div(N, 128));
+    args.k_stages = static_cast<int>(ceil_div(K, kWtK));
+    args.k_split = static_cast<uint32_t>(splits);
+    args.act_box_bytes = act_rows * 128;
+    args.status = status_ptr();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = static_cast<int64_t>(args.t_tiles) * args.w_tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kWtThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if constexpr (SPLIT) {
+        cfg.gridDim = dim3(static_cast<unsigned>(tiles * splits));
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    } else {
+        // 16 dequantizing warps include the epilogue warps: every CTA must own exactly one tile
+        if (DQW == 16 && tiles > sm_count()) return MXQ_ERR_UNSUPPORTED;
+        cfg.gridDim = dim3(static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count()));
+    }
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, tsf, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
+// K splits for a few-tile problem: as many as keep every cluster resident at once (at most
+// max_splits), each split owning at least 2 K stages of 256.
+int w16_splits(int64_t tiles, int64_t k_stages, int max_splits) {
+    int64_t s = sm_count() / (tiles > 0 ? tiles : 1);
+    if (s > max_splits) s = max_splits;
+    if (s > k_stages / 2) s = k_stages / 2;
+    return s < 2 ? 1 : static_cast<int>(s);
+}
+
 template <int FMT, bool F32>
 int dispatch_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w, int64_t M, int64_t N,
                  int64_t K, void* out, cudaStream_t stream) {
-    // More than 128 rows: 256 x 256 tiles, two M=128 MMAs sharing each dequantized W tile.  Up to
-    // 128 rows: 128 x 64 tiles, which gives the most CTAs for the weight stream.
+    // More than 128 tokens: dequantize each 256-row weight tile once into shared memory for two
+    // M=128 MMAs (256 x 256 tiles).  Up to 128 tokens the weight stream dominates: weights go to
+    // TMEM, 256 K per stage, split along K when there are few tiles.
     if (M > 128) return run_w16<FMT, 2, 256, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream);
-    return run_w16<FMT, 1, 64, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream);
+    const int64_t w_tiles = ceil_div(N, 128), k_stages = ceil_div(K, kWtK);
+    // With one tile per CTA (a K split, or no more tiles than SMs) the epilogue warps have nothing
+    // to overlap and dequantize too (16 warps); otherwise 8 warps dequantize while 8 drain.
+    if (M > 32) {
+        const int64_t tiles = w_tiles * ceil_div(M, 64);
+        const int s = w16_splits(tiles, k_stages, 4);
+        if (s > 1) return run_w16t<FMT, 64, 4, 3, true, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, s);
+        return tiles <= sm_count() ? run_w16t<FMT, 64, 4, 3, false, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1)
+                                   : run_w16t<FMT, 64, 4, 3, false, 8, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1);
+    }
+    const int s = w16_splits(w_tiles, k_stages, 4);
+    if (s > 1) return run_w16t<FMT, 32, 6, 3, true, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, s);
+    return w_tiles <= sm_count() ? run_w16t<FMT, 32, 6, 3, false, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1)
+                                 : run_w16t<FMT, 32, 6, 3, false, 8, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1);
 }
 
 }  // namespace
