@@ -85,42 +85,63 @@ __device__ __forceinline__ uint4 dequant8_cvt(uint32_t w, float scale) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// The same on the integer and FMA pipes: the bf16 bit patterns of the E2M1 magnitudes 0, 0.5, 1,
-// 1.5, 2, 3, 4, 6 come from byte-permute lookups (high and low byte tables, 3-bit selectors), the
-// sign bits are moved to bit 15, and a bf16x2 multiply applies the scale s2 = (s, s).  Exact when
-// every product is a normal bf16: the scale lies in [2^-125, 2^125] (MXFP4) or is an E4M3 value
-// (NVFP4; products in [2^-10, 2688]).
-__device__ __forceinline__ uint4 dequant8_prmt(uint32_t w, uint32_t s2) {
-    constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u;  // high bytes of magnitudes 0-3, 4-7
-    constexpr uint32_t kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;  // low bytes
-    const uint32_t m0 = w & 0x77777777u, m1 = m0 >> 16;           // magnitudes as byte selectors (low 16 bits)
-    uint32_t hi0 = __byte_perm(kHiLo, kHiHi, m0), lo0 = __byte_perm(kLoLo, kLoHi, m0);
-    uint32_t hi1 = __byte_perm(kHiLo, kHiHi, m1), lo1 = __byte_perm(kLoLo, kLoHi, m1);
-    // the sign of code i (bit 4i + 3) is bit 7 of byte i / 2 of w << 4 (even i) or of w (odd i)
-    const uint32_t sh = w << 4;
-    hi0 |= __byte_perm(sh, w, 0x5140) & 0x80808080u;
-    hi1 |= __byte_perm(sh, w, 0x7362) & 0x80808080u;
-    const uint32_t p[4] = {__byte_perm(lo0, hi0, 0x5140), __byte_perm(lo0, hi0, 0x7362), __byte_perm(lo1, hi1, 0x5140),
-                           __byte_perm(lo1, hi1, 0x7362)};
-    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+// The same on the integer and FMA pipes.  Codes 2i and 2i+1 of the word are moved to bits 0-3 and
+// 16-19 of one register (byte permute; selector nibbles 8-B yield zero bytes, as the selected bytes
+// have a clear top bit), one integer multiply by 2^6 + 2^12 copies each code to bits 6-9 and 12-15
+// (no carries: the copies do not overlap), and a mask keeps the magnitude bits at 6-8 and the sign
+// at bit 15.  That bf16 pattern s<<15 | m<<6 reads as the code's value times 2^-126 (0.5 is the
+// subnormal 0x0040), so a bf16x2 multiply by f2 = (2^126 s, 2^126 s) yields the scaled elements,
+// exactly whenever every product is a normal bf16.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ uint4 dequant8_mul(uint32_t w, uint32_t f2) {
+    const uint32_t ev = w & 0x0F0F0F0Fu;         // codes 0, 2, 4, 6 in the low nibbles of bytes 0-3
+    const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
+    const uint32_t z[4] = {prmt(ev, od, 0x8480u), prmt(ev, od, 0x9591u), prmt(ev, od, 0xA6A2u), prmt(ev, od, 0xB7B3u)};
+    const __nv_bfloat162 f = *reinterpret_cast<const __nv_bfloat162*>(&f2);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]), sc);
+        const uint32_t t = (z[i] * 0x1040u) & 0x81C081C0u;
+        const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&t), f);
         o[i] = *reinterpret_cast<const uint32_t*>(&v);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// True if the E8M0 codes in the low `n` bytes of `codes` all lie in [2, 252] (scales 2^-125 ..
-// 2^125), where dequant8_prmt is exact.
+// f2 for an MXFP4 block with E8M0 code x: 2^126 * 2^(x - 127) = 2^(x - 1), a normal bf16 for x in
+// [1, 128]; every product is then normal and exact for x in [2, 128].
+__device__ __forceinline__ uint32_t mx_factor2(uint32_t x) { return ((x + 126u) << 7) * 0x10001u; }
+
+// f2 for an NVFP4 block with E4M3 code c: 2^118 times the code's value, so that the dequantized
+// elements are 2^-8 times the NVFP4 values (the epilogue multiplies by 2^8).  The factor lies in
+// [2^109, 2^127) and the products in [2^-18, 10.5]: all exact normal bf16 numbers.
+__device__ __forceinline__ uint32_t nvfp4_factor2(uint32_t c) {
+    const float f = e4m3_decode_pos(c & 0x7Fu) * 0x1p118f;
+    const __nv_bfloat16 h = __float2bfloat16_rn((c & 0x80u) ? -f : f);
+    return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) * 0x10001u;
+}
+
+// Scale applied after the fp32 accumulation: NVFP4 takes back the 2^-8 of its dequantization
+// factor (an exact power-of-two step) before the global scale.
+template <int FMT>
+__device__ __forceinline__ float w16_epilogue(float acc, float g) {
+    return (FMT == MXQ_NVFP4) ? __fmul_rn(__fmul_rn(acc, 256.0f), g) : acc;
+}
+
+// True if the E8M0 codes in the low `n` bytes of `codes` all lie in [2, 128] (scales 2^-125 .. 2),
+// where dequant8_mul is exact.
 __device__ __forceinline__ bool mx_scales_in_range(uint32_t codes, int n) {
     bool ok = true;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         if (i < n) {
             const uint32_t b = (codes >> (8 * i)) & 0xFFu;
-            ok = ok && b >= 2u && b <= 252u;
+            ok = ok && b >= 2u && b <= 128u;
         }
     return ok;
 }
@@ -282,7 +303,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage's W bytes
                 const uint32_t b_s = smem_u32(smem + C::OFF_B + buf * C::B_BYTES);
-                // MXFP4: the byte-permute path unless some scale of the warp's items leaves 2^-125 .. 2^125
+                // MXFP4: the multiply path unless some scale of the warp's items leaves 2^-125 .. 2
                 bool fast = true;
                 if constexpr (FMT != MXQ_NVFP4) {
                     bool mine = true;
@@ -298,21 +319,18 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                     const uint32_t sw = static_cast<uint32_t>(row & 7);
                     uint4 o0, o1, o2, o3;
                     if constexpr (FMT == MXQ_NVFP4) {
-                        // E4M3 block scales (exact in bf16); the first 16 elements take s0, the rest s1
-                        const uint32_t c0 = sc[i] & 0xFFu, c1 = sc[i] >> 8;
-                        const __nv_bfloat16 b0 = __float2bfloat16_rn(e4m3_decode_pos(c0 & 0x7Fu) * ((c0 & 0x80u) ? -1.0f : 1.0f));
-                        const __nv_bfloat16 b1 = __float2bfloat16_rn(e4m3_decode_pos(c1 & 0x7Fu) * ((c1 & 0x80u) ? -1.0f : 1.0f));
-                        const uint32_t u0 = *reinterpret_cast<const uint16_t*>(&b0), u1 = *reinterpret_cast<const uint16_t*>(&b1);
-                        o0 = dequant8_prmt(codes[i].x, u0 * 0x10001u);
-                        o1 = dequant8_prmt(codes[i].y, u0 * 0x10001u);
-                        o2 = dequant8_prmt(codes[i].z, u1 * 0x10001u);
-                        o3 = dequant8_prmt(codes[i].w, u1 * 0x10001u);
+                        // E4M3 block scales; the first 16 elements take s0, the rest s1
+                        const uint32_t f0 = nvfp4_factor2(sc[i] & 0xFFu), f1 = nvfp4_factor2(sc[i] >> 8);
+                        o0 = dequant8_mul(codes[i].x, f0);
+                        o1 = dequant8_mul(codes[i].y, f0);
+                        o2 = dequant8_mul(codes[i].z, f1);
+                        o3 = dequant8_mul(codes[i].w, f1);
                     } else if (fast) {
-                        const uint32_t s2 = (sc[i] << 7) * 0x10001u;  // bf16 2^(code - 127), twice
-                        o0 = dequant8_prmt(codes[i].x, s2);
-                        o1 = dequant8_prmt(codes[i].y, s2);
-                        o2 = dequant8_prmt(codes[i].z, s2);
-                        o3 = dequant8_prmt(codes[i].w, s2);
+                        const uint32_t f = mx_factor2(sc[i]);
+                        o0 = dequant8_mul(codes[i].x, f);
+                        o1 = dequant8_mul(codes[i].y, f);
+                        o2 = dequant8_mul(codes[i].z, f);
+                        o3 = dequant8_mul(codes[i].w, f);
                     } else {
                         const float s = pow2f(static_cast<int>(sc[i]) - 127);
                         o0 = dequant8_cvt(codes[i].x, s);
@@ -366,22 +384,22 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                             float4* dst = reinterpret_cast<float4*>(orow + nb);
 #pragma unroll
                             for (int v = 0; v < 8; ++v)
-                                dst[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
-                                                     __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                                     __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                                     __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+                                dst[v] = make_float4(w16_epilogue<FMT>(__uint_as_float(r[4 * v]), alpha),
+                                                     w16_epilogue<FMT>(__uint_as_float(r[4 * v + 1]), alpha),
+                                                     w16_epilogue<FMT>(__uint_as_float(r[4 * v + 2]), alpha),
+                                                     w16_epilogue<FMT>(__uint_as_float(r[4 * v + 3]), alpha));
                         } else {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
-                                if (nb + i < p.N) orow[nb + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                                if (nb + i < p.N) orow[nb + i] = w16_epilogue<FMT>(__uint_as_float(r[i]), alpha);
                         }
                     } else {
                         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                                           __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                            const __nv_bfloat162 b = __floats2bfloat162_rn(w16_epilogue<FMT>(__uint_as_float(r[2 * i]), alpha),
+                                                                           w16_epilogue<FMT>(__uint_as_float(r[2 * i + 1]), alpha));
                             packed[i] = *reinterpret_cast<const uint32_t*>(&b);
                         }
                         if ((p.N & 7) == 0 && nb + 32 <= p.N) {
@@ -435,6 +453,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 // persistent over tiles (tokens fastest) with two accumulators when TMEM has room.
 
 constexpr int kWtDeqWarps = 8;  // 16 (the epilogue warps too) when every CTA owns one tile
+constexpr int kWtGroups16 = 2;  // 16 dequantizing warps form this many groups taking turns on stages
 constexpr int kWtEpiWarps = 8;
 constexpr int kWtThreads = (2 + kWtDeqWarps + kWtEpiWarps) * 32;
 constexpr int kWtK = 256;  // K elements per stage
@@ -480,6 +499,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     w4a16_tmem_kernel(const __grid_constant__ CUtensorMap tma_act, const __grid_constant__ CUtensorMap tma_w,
                       const __grid_constant__ CUtensorMap tma_sf, const W16TArgs p) {
     using C = W16TCfg<FMT, NT, STAGES, AS, SPLIT>;
+    constexpr int GROUPS = DQW == 16 ? kWtGroups16 : 1;  // dequantizing warp groups, taking turns on stages
+    constexpr int WPS = DQW / GROUPS;                    // dequantizing warps per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // activations, codes, scales landed
@@ -502,10 +523,10 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         prefetch_tmap(&tma_sf);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + DQW);
+            mbar_init(&empty[s], 1 + WPS);
         }
         for (int a = 0; a < AS; ++a) {
-            mbar_init(&aready[a], DQW);
+            mbar_init(&aready[a], WPS);
             mbar_init(&aempty[a], 1);
         }
         for (int b = 0; b < C::ACC; ++b) {
@@ -609,16 +630,19 @@ __global__ void __launch_bounds__(kWtThreads, 1)
             }
         }
     } else if (warp < 2 + DQW) {
-        // dequantization: this thread's weight row of the tile is its TMEM lane; warp group kq
-        // converts K elements [KE * kq, + KE) of the stage (KE / 2 bytes of codes, NBLK scale blocks)
-        // into TMEM columns [KE / 2 * kq, + KE / 2) of the slot, 64 elements at a time
-        constexpr int KE = 4 * kWtK / DQW;   // 128 or 64
+        // dequantization: this thread's weight row of the tile is its TMEM lane; in the stages of
+        // its group, warp quad kq converts K elements [KE * kq, + KE) (KE / 2 bytes of codes, NBLK
+        // scale blocks) into TMEM columns [KE / 2 * kq, + KE / 2) of the slot, 64 elements at a time.
+        // Groups taking turns keep one group's shared-memory loads and waits under another's math.
+        constexpr int KE = 4 * kWtK / WPS;   // 128 or 64
         constexpr int NCH = KE / 32;         // 16-byte code pieces per thread
         constexpr int NBLK = KE / C::BS;     // scale blocks per thread
         constexpr int NSW = (NBLK + 3) / 4;  // 32-bit scale words per thread
         const int r = 32 * (warp & 3) + lane;
-        const int kq = (warp - 2) >> 2;
+        const int kq = ((warp - 2) % WPS) >> 2;
+        const int grp = (warp - 2) / WPS;
         const int blk0 = NBLK * kq;  // the warp's first scale block in the stage
+        int turn = 0;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const uint32_t sw = static_cast<uint32_t>(r & 7);  // 128-byte swizzle of the code rows
         int stage = 0, slot = 0;
@@ -626,83 +650,81 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         bool ok = true;
         for (int tile = first; tile < num_tiles && ok; tile += step) {
             for (int ks = k0; ks < k1; ++ks) {
-                if (!mbar_wait_warp(&full[stage], phase, p.status, 55)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t w_row = smem_u32(smem + C::OFF_W + stage * C::W_BYTES) + r * 128;
-                uint4 c[NCH];
+                const bool mine = GROUPS == 1 || turn == grp;
+                if (++turn == GROUPS) turn = 0;
+                if (mine) {
+                    if (!mbar_wait_warp(&full[stage], phase, p.status, 55)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t w_row = smem_u32(smem + C::OFF_W + stage * C::W_BYTES) + r * 128;
+                    uint4 c[NCH];
 #pragma unroll
-                for (int q = 0; q < NCH; ++q) c[q] = ld_shared_v4(w_row + (((NCH * kq + q) ^ sw) << 4));
-                // a 512-byte scale tile holds 4 consecutive blocks of each of the 128 rows
-                const uint32_t sf_row = smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES) + (r & 31) * 16 + (r >> 5) * 4;
-                uint32_t sc[NSW];
+                    for (int q = 0; q < NCH; ++q) c[q] = ld_shared_v4(w_row + (((NCH * kq + q) ^ sw) << 4));
+                    // a 512-byte scale tile holds 4 consecutive blocks of each of the 128 rows
+                    const uint32_t sf_row = smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES) + (r & 31) * 16 + (r >> 5) * 4;
+                    uint32_t sc[NSW];
 #pragma unroll
-                for (int i = 0; i < NSW; ++i)
-                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc[i]) : "r"(sf_row + ((blk0 >> 2) + i) * 512));
-                if constexpr (NBLK < 4) sc[0] >>= 8 * (blk0 & 3);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage's codes and scales
-                if (!mbar_wait_warp(&aempty[slot], sphase ^ 1u, p.status, 56)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t t_col =
-                    tmem_base + lane_addr + static_cast<uint32_t>(C::A_TMEM + slot * 128 + kq * (KE / 2));
-                // MXFP4: the byte-permute path unless some scale of the warp leaves 2^-125 .. 2^125
-                const bool fast = (FMT == MXQ_NVFP4) || __all_sync(0xFFFFFFFFu, mx_scales_in_range(sc[0], NBLK));
-                if (fast) {
-                    uint32_t s2[NBLK];  // block scales as bf16x2 (s, s)
+                    for (int i = 0; i < NSW; ++i)
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc[i]) : "r"(sf_row + ((blk0 >> 2) + i) * 512));
+                    if constexpr (NBLK < 4) sc[0] >>= 8 * (blk0 & 3);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage's codes and scales
+                    if (!mbar_wait_warp(&aempty[slot], sphase ^ 1u, p.status, 56)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t t_col =
+                        tmem_base + lane_addr + static_cast<uint32_t>(C::A_TMEM + slot * 128 + kq * (KE / 2));
+                    // MXFP4: the multiply path unless some scale of the warp leaves 2^-125 .. 2
+                    const bool fast = (FMT == MXQ_NVFP4) || __all_sync(0xFFFFFFFFu, mx_scales_in_range(sc[0], NBLK));
+                    if (fast) {
+                        uint32_t f2[NBLK];  // per-block dequantization factors
 #pragma unroll
-                    for (int b = 0; b < NBLK; ++b) {
-                        const uint32_t code = (sc[b >> 2] >> (8 * (b & 3))) & 0xFFu;
-                        if constexpr (FMT == MXQ_NVFP4) {
-                            const __nv_bfloat16 h =
-                                __float2bfloat16_rn(e4m3_decode_pos(code & 0x7Fu) * ((code & 0x80u) ? -1.0f : 1.0f));
-                            s2[b] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) * 0x10001u;
-                        } else {
-                            s2[b] = (code << 7) * 0x10001u;  // bf16 2^(code - 127)
+                        for (int b = 0; b < NBLK; ++b) {
+                            const uint32_t code = (sc[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+                            f2[b] = (FMT == MXQ_NVFP4) ? nvfp4_factor2(code) : mx_factor2(code);
+                        }
+#pragma unroll
+                        for (int hq = 0; hq < KE / 64; ++hq) {  // 64 elements (two 16-byte code pieces) at a time
+                            uint32_t v[32];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int wi = 8 * hq + j;  // word index in this warp's KE elements
+                                const uint4 cc = c[wi >> 2];
+                                const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
+                                const uint4 o = dequant8_mul(word, f2[wi * 8 / C::BS]);
+                                v[4 * j + 0] = o.x;
+                                v[4 * j + 1] = o.y;
+                                v[4 * j + 2] = o.z;
+                                v[4 * j + 3] = o.w;
+                            }
+                            tmem_st_cols<32>(t_col + hq * 32, v);
+                        }
+                    } else {
+#pragma unroll
+                        for (int hq = 0; hq < KE / 64; ++hq) {
+                            uint32_t v[32];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int wi = 8 * hq + j;
+                                const uint4 cc = c[wi >> 2];
+                                const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
+                                const uint32_t code = (sc[0] >> (8 * (wi >> 2))) & 0xFFu;
+                                const uint4 o = dequant8_cvt(word, pow2f(static_cast<int>(code) - 127));
+                                v[4 * j + 0] = o.x;
+                                v[4 * j + 1] = o.y;
+                                v[4 * j + 2] = o.z;
+                                v[4 * j + 3] = o.w;
+                            }
+                            tmem_st_cols<32>(t_col + hq * 32, v);
                         }
                     }
-#pragma unroll
-                    for (int hq = 0; hq < KE / 64; ++hq) {  // 64 elements (two 16-byte code pieces) at a time
-                        uint32_t v[32];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int wi = 8 * hq + j;  // word index in this warp's KE elements
-                            const uint4 cc = c[wi >> 2];
-                            const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
-                            const uint4 o = dequant8_prmt(word, s2[wi * 8 / C::BS]);
-                            v[4 * j + 0] = o.x;
-                            v[4 * j + 1] = o.y;
-                            v[4 * j + 2] = o.z;
-                            v[4 * j + 3] = o.w;
-                        }
-                        tmem_st_cols<32>(t_col + hq * 32, v);
-                    }
-                } else {
-#pragma unroll
-                    for (int hq = 0; hq < KE / 64; ++hq) {
-                        uint32_t v[32];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int wi = 8 * hq + j;
-                            const uint4 cc = c[wi >> 2];
-                            const uint32_t word = (wi & 3) == 0 ? cc.x : (wi & 3) == 1 ? cc.y : (wi & 3) == 2 ? cc.z : cc.w;
-                            const uint32_t code = (sc[0] >> (8 * (wi >> 2))) & 0xFFu;
-                            const uint4 o = dequant8_cvt(word, pow2f(static_cast<int>(code) - 127));
-                            v[4 * j + 0] = o.x;
-                            v[4 * j + 1] = o.y;
-                            v[4 * j + 2] = o.z;
-                            v[4 * j + 3] = o.w;
-                        }
-                        tmem_st_cols<32>(t_col + hq * 32, v);
-                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aready[slot]);
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&aready[slot]);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -725,7 +747,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     auto store = [&](int tt, int wt, int j, float val) {
         const int tok = tt * NT + half * HC + j, n = wt * 128 + sub * 32 + lane;
         if (tok < p.M && n < p.N) {
-            const float y = __fmul_rn(val, alpha);
+            const float y = w16_epilogue<FMT>(val, alpha);
             if constexpr (OUT_F32)
                 static_cast<float*>(p.out)[static_cast<int64_t>(tok) * p.N + n] = y;
             else

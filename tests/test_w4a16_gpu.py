@@ -88,13 +88,16 @@ def test_w4a16_scale_placement(fmt, M):
     check_fp32(gpu, ref, abs_sum, "%s scales" % fmt)
 
 
-@pytest.mark.parametrize("codes,a_scale", [((0, 1, 2, 3, 4), 2.0 ** 100), ((248, 249, 250, 251, 252), 2.0 ** -100)])
-def test_w4a16_extreme_mx_scales(codes, a_scale):
-    """E8M0 scales at the ends of the range: 2^-127 and 2^-126 dequantize through the exact fp32
-    path (bf16 subnormal products), 2^-125 ... 2^125 through the byte-permute path.  Activations
-    are scaled so that the products and sums stay normal fp32 numbers."""
-    M, N, K = 130, 96, 256
-    rng = np.random.default_rng(codes[0])
+@pytest.mark.parametrize("M", [130, 32, 100])
+@pytest.mark.parametrize("codes,a_scale", [((0, 1, 2, 3, 4), 2.0 ** 100), ((248, 249, 250, 251, 252), 2.0 ** -100),
+                                           ((126, 127, 128, 129, 130), 1.0), ((2, 3, 127, 128), 1.0)])
+def test_w4a16_extreme_mx_scales(M, codes, a_scale):
+    """E8M0 scales across the range: codes 2 ... 128 (2^-125 ... 2) dequantize through the integer
+    multiply path, the others through the exact fp32 path, chosen per warp; every M covers another
+    kernel (one dequantizing into shared memory, two into tensor memory).  Activations are scaled
+    so that the products and sums stay normal fp32 numbers."""
+    N, K = 96, 256
+    rng = np.random.default_rng(codes[0] + M)
     A = (synth.random_bf16((M, K), 61).float() * a_scale).to(torch.bfloat16)
     Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
     Wsf = rng.choice(np.array(codes, np.uint8), (N, K // 32)).astype(np.uint8)
