@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--no-others", action="store_true", help="skip the informational other-problem timings")
     ap.add_argument("--M", type=int, default=None, help="override the workload's M (profiling runs)")
     ap.add_argument("--N", type=int, default=None, help="override the workload's N (profiling runs)")
+    ap.add_argument("--op", default="linear", choices=["linear", "w4a16"],
+                    help="w4a16: time only the weight-only GEMM on the workload's shape (profiling runs; "
+                         "prints its own JSON line, not the benchmark line)")
+    ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4"], help="weight format of --op w4a16")
     return ap.parse_args()
 
 
@@ -491,8 +495,39 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_w4a16_op(args):
+    """Weight-only GEMM alone: bf16 activations of the workload's shape times its weights quantized
+    to --fmt, timed warm (back-to-back launches) and with the L2 flushed before each launch."""
+    from nvfp4_block_scaled_mx_b200 import mxq
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --op w4a16 needs a CUDA device (there is no CPU fallback)")
+    cfg = synth.CONFIGS[args.workload]
+    M, N, K = args.M or cfg["M"], args.N or cfg["N"], cfg["K"]
+    A = synth.random_bf16((M, K), 71, device="cuda")
+    W = synth.random_bf16((N, K), 72, std=0.02, device="cuda")
+    g_w = mxq.global_scale(W)[0] if args.fmt == "nvfp4" else None
+    W_q, W_sf = mxq.quantize(W, args.fmt, "even", global_scale=g_w)
+    del W
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    f = lambda: mxq.gemm_w4a16(A, W_q, W_sf, N, args.fmt, g_W=g_w, out=out, stream=stream)
+    for _ in range(max(3, args.warmup)):
+        f()
+    warm = time_loop(f, args.steps, stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    cold = time_flushed(f, max(3, args.steps), stream, flush)
+    wbytes = W_q.numel() + W_sf.numel()
+    return {"op": "w4a16", "workload": args.workload, "M": M, "N": N, "K": K, "fmt": args.fmt,
+            "warm_ms": round(warm * 1e3, 4), "l2_flushed_ms": round(cold * 1e3, 4),
+            "tflops_warm": round(2.0 * M * N * K / warm / 1e12, 1),
+            "weight_gbs_l2_flushed": round(wbytes / cold / 1e9, 1)}
+
+
 def main():
     args = parse()
+    if args.op == "w4a16":
+        print(json.dumps(run_w4a16_op(args)), flush=True)
+        return
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":
