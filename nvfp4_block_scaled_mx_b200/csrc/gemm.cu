@@ -430,6 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* empty = full + STAGES;
     uint64_t* sfready = empty + STAGES;
     uint64_t* accf = sfready + STAGES;
+    uint64_t* rready = accf + 1;  // non-leaders: the leader's operand ring is free for the partials
+    uint64_t* rfull = accf + 2;   // leader: every partial has landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -448,6 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sfready[s], kSfWarps);
         }
         mbar_init(accf, 1);
+        mbar_init(rready, 1);
+        mbar_init(rfull, 1);
+        // the partials of rows < M from the other splits-1 CTAs, counted in bytes
+        if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * static_cast<uint32_t>(min(p.M, 128)) * BN * 4);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -457,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    cluster_arrive_relaxed();
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();
 
@@ -559,15 +566,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
-    // reduction: every CTA's epilogue warps hold their share of the partial tile in registers
+    // reduction: every CTA's epilogue warps take their share of the partial tile into registers.
+    // The leader frees its operand ring for the partials once its MMAs are done (a remote arrive
+    // per other CTA); the others send their rows < M with st.async, counted in bytes on the
+    // leader's barrier, and leave.  Layout in the leader: [splits-1][BN/4 column quads][128 rows][4]
+    // fp32, so that the 32 rows of a warp move 512 contiguous bytes per 16-byte access.
     constexpr int COLS = BN / 2;
     const bool epi = warp >= 2 && warp < 2 + kEpiWarps;
     const int sub = warp & 3;
     const int col0 = ((warp - 2) >> 2) * COLS;
     const int row = sub * 32 + lane;
+    float* red = reinterpret_cast<float*>(smem);
     float acc[COLS];
+    cluster_wait();  // every CTA of the cluster has initialised its barriers
     if (epi) {
         const bool ok = mbar_wait(accf, 0, p.status, 24);
+        if (split == 0 && warp == 2 && lane == 0)
+            for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
         tc_fence_after();
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
 #pragma unroll
@@ -580,25 +595,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
     }
-    // 1: every CTA's MMAs are done, so the leader's operand ring is free for the partials
-    __syncthreads();
-    cluster_sync();
-    float* red = reinterpret_cast<float*>(smem);  // leader: [splits-1][128 rows][BN] fp32
-    if (epi && split != 0 && row < p.M) {
-        const uint32_t dst = mapa_shared(smem_u32(red + ((split - 1) * 128 + row) * BN + col0), 0);
+    if (epi && split != 0 && row < p.M && mbar_wait_cluster(rready, 0, p.status, 27)) {
+        const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (BN / 4) + col0 / 4) * 128 + row) * 4), 0);
+        const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
 #pragma unroll
         for (int v = 0; v < COLS / 4; ++v)
-            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + v * 16), "f"(acc[4 * v]),
-                         "f"(acc[4 * v + 1]), "f"(acc[4 * v + 2]), "f"(acc[4 * v + 3])
-                         : "memory");
+            st_async_v4(dst + v * 128 * 16, acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3], bar);
     }
-    // 2: all partials sit in the leader's shared memory
-    cluster_sync();
     if (epi && split == 0 && row < p.M) {
-        for (uint32_t sp = 1; sp < splits; ++sp) {
-            const float* src = red + ((sp - 1) * 128 + row) * BN + col0;
+        const bool got = mbar_wait(rfull, 0, p.status, 28);
+        for (uint32_t sp = 1; got && sp < splits; ++sp) {
+            const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (BN / 4) + col0 / 4) * 128 + row;
 #pragma unroll
-            for (int i = 0; i < COLS; ++i) acc[i] = __fadd_rn(acc[i], src[i]);
+            for (int v = 0; v < COLS / 4; ++v) {
+                const float4 q = src[v * 128];
+                acc[4 * v] = __fadd_rn(acc[4 * v], q.x);
+                acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], q.y);
+                acc[4 * v + 2] = __fadd_rn(acc[4 * v + 2], q.z);
+                acc[4 * v + 3] = __fadd_rn(acc[4 * v + 3], q.w);
+            }
         }
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
         const int n0 = nt * BN + col0;

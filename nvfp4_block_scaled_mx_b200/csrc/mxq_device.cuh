@@ -74,6 +74,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     }
 }
 
+// mbar_wait with cluster-scope acquire, for a phase completed by a release arrive from another CTA
+// of the cluster.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status, int where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((n & 63u) == 0 && globaltimer() - t0 > kWaitLimitNs) {
+            if (status) atomicCAS(status, 0, kStatusTimeoutBase + where);
+            return false;
+        }
+    }
+}
+
 // The same wait by every lane of a converged warp, with one decision for the warp: a timeout in
 // any lane aborts all of them, so the warp never splits around a later warp-wide operation.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, int where) {
@@ -368,6 +394,24 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 // All threads of both CTAs of the cluster.
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Split cluster barrier: arrive once after the mbarrier initialisation (fenced at cluster scope),
+// wait before the first access to another CTA's shared memory.  The wait then only confirms that
+// every CTA of the cluster has started and initialised its barriers.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// 16 bytes from registers into another CTA's shared memory (cluster address), counted as
+// complete_tx bytes on an mbarrier of that CTA (cluster address).
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                            uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     cluster_addr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
+                 : "memory");
 }
 
 // shared::cluster address of the variable at this CTA-local shared address in CTA `rank`.

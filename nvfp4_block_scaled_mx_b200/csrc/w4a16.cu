@@ -474,11 +474,12 @@ struct W16TCfg {
     static constexpr int OFF_W = OFF_ACT + STAGES * ACT_BYTES;
     static constexpr int OFF_SF = OFF_W + STAGES * W_BYTES;
     static constexpr int OFF_BAR = OFF_SF + STAGES * SF_BYTES;
-    static constexpr int N_BARS = 2 * STAGES + 2 * AS + 2 * ACC;
+    static constexpr int N_BARS = 2 * STAGES + 2 * AS + 2 * ACC + 2;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N");
     static_assert(COLS_USED <= 512, "TMEM budget");
+    static_assert(!SPLIT || 3 * 128 * NT * 4 <= OFF_BAR, "split-K partials fit below the barriers");
     static_assert(ACT_SUB % 1024 == 0, "128B-swizzled activation boxes stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -509,6 +510,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     uint64_t* aempty = aready + AS;                                    // MMAs done with the weight slot
     uint64_t* accf = aempty + AS;                                      // accumulator ready
     uint64_t* acce = accf + C::ACC;                                    // accumulator drained
+    uint64_t* rready = acce + C::ACC;  // split, non-leaders: the leader's operand ring is free for the partials
+    uint64_t* rfull = rready + 1;      // split, leader: every partial has landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -533,6 +536,12 @@ __global__ void __launch_bounds__(kWtThreads, 1)
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], kWtEpiWarps);
         }
+        if constexpr (SPLIT) {
+            mbar_init(rready, 1);
+            mbar_init(rfull, 1);
+            // the other splits-1 CTAs' partial tiles, counted in bytes
+            if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * 128u * NT * 4u);
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -542,6 +551,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if constexpr (SPLIT) cluster_arrive_relaxed();
     const uint32_t tmem_base = *tmem_slot;
 
     // tiles: tokens fastest; a SPLIT cluster takes one tile and a contiguous range of K stages
@@ -784,10 +794,19 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         tc_fence_before();
         __syncthreads();
     } else {
-        // every CTA's epilogue warps take their partial tile into registers
+        // every CTA's epilogue warps take their partial tile into registers.  The leader frees its
+        // operand ring once its MMAs are done (a remote arrive per other CTA); the others send their
+        // partials with st.async, counted in bytes on the leader's barrier, and leave.  Layout in
+        // the leader: [splits-1][NT/4 column quads][128 rows][4] fp32, so that the 32 rows of a warp
+        // move 512 contiguous bytes per 16-byte access.
         float part[HC];
+        float* red = reinterpret_cast<float*>(smem);
+        const int row = sub * 32 + lane;
+        cluster_wait();  // every CTA of the cluster has initialised its barriers
         if (epi) {
             const bool ok = mbar_wait(&accf[0], 0, p.status, 58);
+            if (split == 0 && warp == 2 + kWtDeqWarps && lane == 0)
+                for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(half * HC);
 #pragma unroll
@@ -800,27 +819,28 @@ __global__ void __launch_bounds__(kWtThreads, 1)
             }
             tc_fence_before();
         }
-        // 1: every CTA's MMAs are done, so the leader's operand ring is free for the partials
-        __syncthreads();
-        cluster_sync();
-        float* red = reinterpret_cast<float*>(smem);  // leader: [splits-1][128 rows][NT] fp32
-        const int row = sub * 32 + lane;
-        if (epi && split != 0) {
-            const uint32_t dst = mapa_shared(smem_u32(red + ((split - 1) * 128 + row) * NT + half * HC), 0);
+        if (epi && split != 0 && mbar_wait_cluster(rready, 0, p.status, 59)) {
+            const uint32_t dst =
+                mapa_shared(smem_u32(red + (((split - 1) * (NT / 4) + half * HC / 4) * 128 + row) * 4), 0);
+            const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
 #pragma unroll
             for (int v4 = 0; v4 < HC / 4; ++v4)
-                asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + v4 * 16), "f"(part[4 * v4]),
-                             "f"(part[4 * v4 + 1]), "f"(part[4 * v4 + 2]), "f"(part[4 * v4 + 3])
-                             : "memory");
+                st_async_v4(dst + v4 * 128 * 16, part[4 * v4], part[4 * v4 + 1], part[4 * v4 + 2], part[4 * v4 + 3],
+                            bar);
         }
-        // 2: all partials sit in the leader's shared memory
-        cluster_sync();
         if (epi && split == 0) {
             const int tt = first % p.t_tiles, wt = first / p.t_tiles;
-            for (uint32_t sp = 1; sp < splits; ++sp) {
-                const float* src = red + ((sp - 1) * 128 + row) * NT + half * HC;
+            const bool got = mbar_wait(rfull, 0, p.status, 60);
+            for (uint32_t sp = 1; got && sp < splits; ++sp) {
+                const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (NT / 4) + half * HC / 4) * 128 + row;
 #pragma unroll
-                for (int j = 0; j < HC; ++j) part[j] = __fadd_rn(part[j], src[j]);
+                for (int v4 = 0; v4 < HC / 4; ++v4) {
+                    const float4 q = src[v4 * 128];
+                    part[4 * v4] = __fadd_rn(part[4 * v4], q.x);
+                    part[4 * v4 + 1] = __fadd_rn(part[4 * v4 + 1], q.y);
+                    part[4 * v4 + 2] = __fadd_rn(part[4 * v4 + 2], q.z);
+                    part[4 * v4 + 3] = __fadd_rn(part[4 * v4 + 3], q.w);
+                }
             }
 #pragma unroll
             for (int j = 0; j < HC; ++j) store(tt, wt, j, part[j]);
