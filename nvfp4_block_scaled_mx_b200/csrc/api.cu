@@ -197,7 +197,7 @@ int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_
         return MXQ_ERR_ALIGN;
     if ((rc = check_device()) != MXQ_OK) return rc;
     return launch_gemm(A_q, A_sf, B_q, B_sf, g_A, g_B, M, N, K, fmt, out_type, out,
-                       reinterpret_cast<cudaStream_t>(stream), false);
+                       reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
@@ -236,6 +236,9 @@ int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const f
     uint8_t* a_q = static_cast<uint8_t*>(workspace);
     uint8_t* a_sf = a_q + round256(qb);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // few tokens: one launch, the GEMM quantizing its own activations (the workspace stays unused)
+    rc = launch_linear_fused(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, out, st);
+    if (rc != kNotFused) return rc;
     if (launch_quantize(x_bf16, M, K, fmt, act_rule, g_A, a_q, a_sf, MXQ_SF_SWIZZLED, st) != cudaSuccess)
         return MXQ_ERR_CUDA;
     return launch_gemm(a_q, a_sf, W_q, W_sf, g_A, g_W, M, N, K, fmt, out_type, out, st, true);

@@ -26,6 +26,7 @@
 
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
+#include "quant_block.cuh"
 
 namespace mxq {
 
@@ -94,7 +95,8 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
     static constexpr int N_BARS = 3 * STAGES + 2 * ACC_STAGES;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int OFF_TAB = OFF_SLOT + 16;             // NVFP4 d and 1/d tables (in-kernel quantizer)
+    static constexpr int SMEM_BYTES = OFF_TAB + 1024 + 1024;  // + slack for 1024-byte alignment
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -112,6 +114,7 @@ struct GemmArgs {
     uint32_t k_split;      // split-K kernel: CTAs per cluster sharing one output tile
     uint32_t a_box_bytes;  // split-K kernel: bytes of one A load (rows rounded up to 8, <= 128)
     uint32_t tma_store;    // pair kernel: bf16 output written through TMA stores (N % 8 == 0)
+    const void* x;         // split-K kernel quantizing its own A: the bf16 activations [M, K]
 };
 
 template <int KIND, int BN, int STAGES, bool OUT_F32>
@@ -154,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // operands may come from the kernel launched just before this one on the stream
     pdl_wait();
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     const int num_tiles = p.m_tiles * p.n_tiles;
     auto groups_of = [&](int tile) {
@@ -417,11 +421,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr uint32_t kMaxSplits = 4;
 
-template <int KIND, bool OUT_F32>
+// QRULE >= 0 (M <= 32): A is not pre-quantized.  TMA brings the stage's bf16 activations (boxes of
+// 64 elements x rows, 128B swizzle; at most 32 rows x BK x 2 bytes = the stage's A buffer) and the
+// scale-staging warps quantize them in place into the A tile and the A scale tiles (rule QRULE for
+// MX formats) with the streaming quantizer's arithmetic, so a few-token linear layer is one launch.
+template <int KIND, bool OUT_F32, int QRULE = -1>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                        const GemmArgs p) {
     constexpr int BN = 128, STAGES = 6;
+    constexpr bool QA = QRULE >= 0;
     using C = Cfg<KIND, BN, STAGES>;
     static_assert((kMaxSplits - 1) * 128 * BN * 4 <= STAGES * (C::A_BYTES + C::B_BYTES), "reduction buffer");
     extern __shared__ uint8_t smem_raw[];
@@ -466,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_arrive_relaxed();
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     const bool b_group = nt < p.b_row_tiles;  // always true: one 128-row B group per tile
     if (warp == 0) {
@@ -478,11 +488,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (elect_one()) {
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
                 // A rows past M are not loaded: they only feed accumulator rows that are never stored
-                mbar_arrive_expect_tx(&full[stage], p.a_box_bytes + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
-                tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES, ks * 128, 0, pol);
+                constexpr int A_BOXES = QA ? C::BK / 64 : 1;  // bf16 boxes of 64 elements, or one FP4/FP8 box
+                mbar_arrive_expect_tx(&full[stage], A_BOXES * p.a_box_bytes + C::B_BYTES +
+                                                        atoms * 512 * ((QA ? 0 : 1) + (b_group ? 1 : 0)));
+#pragma unroll
+                for (int b = 0; b < A_BOXES; ++b)
+                    tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES + b * p.a_box_bytes,
+                                (QA ? ks * C::BK * 2 : ks * 128) + b * 128, 0, pol);
                 tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, nt * BN, pol);
                 const int64_t kcol = static_cast<int64_t>(ks) * C::SF_ATOMS;
-                bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, p.a_sf + kcol * 512, atoms * 512, &full[stage]);
+                if (!QA)
+                    bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, p.a_sf + kcol * 512, atoms * 512, &full[stage]);
                 if (b_group)
                     bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES,
                               p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + kcol) * 512, atoms * 512,
@@ -531,14 +547,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && elect_one()) tc_commit(accf);
         __syncwarp();
-    } else if (warp >= 2 + kEpiWarps) {
+    } else if (warp >= 2 + kEpiWarps || (QA && warp >= 6 && warp < 2 + kEpiWarps)) {
+        // scale staging (warps 10-13, one per TMEM sub-partition).  With the in-kernel quantizer
+        // epilogue warps 6-9 (again one per sub-partition) form a second group, and the two groups
+        // take alternate stages, so that one group's barrier and load latencies sit under the other's
         const int sub = warp & 3;
         const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+        const int grp = warp >= 2 + kEpiWarps ? 0 : 1;
+        const int bar_id = 1 + grp;
         int stage = 0;
         uint32_t phase = 0;
+        // in-kernel quantizer: thread qt of the group's 4 warps takes units (row, j) of 32 elements
+        const int qt = (warp & 3) * 32 + lane;
+        constexpr int UPR = C::BK / 32;  // 32-element units per row and stage
+        constexpr int UPT = 32 * UPR / 128;  // units per thread at most (M <= 32)
+        float* tab_d = reinterpret_cast<float*>(smem + C::OFF_TAB);
+        float* tab_r = tab_d + 128;
+        float g_a = 1.0f;
+        if constexpr (QA && KIND == 1) {
+            g_a = *p.g_a;
+            const float d = __fmul_rn(e4m3_decode_pos(static_cast<uint32_t>(qt)), g_a);
+            tab_d[qt] = d;
+            tab_r[qt] = d == 0.0f ? 0.0f : __frcp_rn(d);  // both groups write the same values
+            named_barrier_sync(bar_id, 4 * 32);
+        }
         for (int ks = k0; ks < k1; ++ks) {
-            if (!mbar_wait(&full[stage], phase, p.status, 26)) break;
+            if (QA && ((ks - k0) & 1) != grp) {
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                continue;
+            }
+            if constexpr (QA) {
+                if (named_barrier_or(bar_id, 4 * 32, !mbar_wait(&full[stage], phase, p.status, 26))) break;
+                const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                uint8_t* sfa = smem + C::OFF_SFA + stage * C::SFA_BYTES;
+                // read this thread's units of bf16 (unit (row, j) = 64 bytes of box j / 2) ...
+                uint32_t w[UPT][16];
+#pragma unroll
+                for (int u = 0; u < UPT; ++u) {
+                    const int v = qt + u * 128, row = v / UPR, jj = v - row * UPR;
+                    if (row < p.M && static_cast<int64_t>(ks) * C::BK + jj * 32 < p.K) {
+                        const uint32_t rb = a_s + (jj >> 1) * p.a_box_bytes + row * 128;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 t = ld_shared_v4(rb + ((((jj & 1) * 4 + i) ^ (row & 7)) << 4));
+                            w[u][4 * i] = t.x;
+                            w[u][4 * i + 1] = t.y;
+                            w[u][4 * i + 2] = t.z;
+                            w[u][4 * i + 3] = t.w;
+                        }
+                    }
+                }
+                named_barrier_sync(bar_id, 4 * 32);  // ... before any thread overwrites the buffer with codes
+#pragma unroll
+                for (int u = 0; u < UPT; ++u) {
+                    const int v = qt + u * 128, row = v / UPR, j = v - row * UPR;
+                    if (row >= p.M || static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
+                    uint32_t codes[8], seen = 0;
+                    const uint32_t sc =
+                        quantize32<KIND, (QRULE < 0 ? 0 : QRULE), false>(w[u], g_a, tab_d, tab_r, codes, seen);
+                    const uint32_t sw = static_cast<uint32_t>(row & 7);
+                    const uint32_t sf_row = (row & 31) * 16 + ((row >> 5) & 3) * 4;
+                    const uint32_t a_row = a_s + row * 128;
+                    if constexpr (KIND == 2) {  // MXFP8: 32 bytes of codes, one scale block
+                        st_shared_v4(a_row + (((2 * j) ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                        st_shared_v4(a_row + (((2 * j + 1) ^ sw) << 4), make_uint4(codes[4], codes[5], codes[6], codes[7]));
+                        sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
+                    } else if constexpr (KIND == 1) {  // NVFP4: 16 bytes of codes, scale blocks 2j and 2j + 1
+                        st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                        *reinterpret_cast<uint16_t*>(sfa + ((2 * j) >> 2) * 512 + sf_row + ((2 * j) & 3)) =
+                            static_cast<uint16_t>(sc);
+                    } else {  // MXFP4: 16 bytes of codes, one scale block
+                        st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                        sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
+                    }
+                }
+                fence_proxy_async_smem();            // the A tile is read next by the tensor cores
+                named_barrier_sync(bar_id, 4 * 32);  // every scale byte of the stage is in shared memory
+            } else if (!mbar_wait(&full[stage], phase, p.status, 26)) {
+                break;
+            }
             uint32_t r[C::SF_COLS_STAGE];
+
             const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES) + lane * 16;
             const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES) + lane * 16;
 #pragma unroll
@@ -762,6 +854,7 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     pdl_wait();
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     const int m_tiles = (p.M + 255) / 256;
     const int num_tiles = m_tiles * p.n_tiles;
@@ -1151,14 +1244,18 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
     return MXQ_OK;
 }
 
-template <int KIND, bool F32>
+template <int KIND, bool F32, int QRULE = -1>
 int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cudaStream_t stream, bool pdl) {
     using C = Cfg<KIND, 128, 6>;
-    auto kern = gemm_splitk_kernel<KIND, F32>;
+    auto kern = gemm_splitk_kernel<KIND, F32, QRULE>;
     const int row_bytes = args.K / C::EPB;
     CUtensorMap ta, tb;
     const uint32_t a_rows = static_cast<uint32_t>(ceil_div(args.M, 8) * 8);
-    if (!make_map(&ta, A_q, row_bytes, args.M, a_rows) || !make_map(&tb, B_q, row_bytes, args.N, 128)) return MXQ_ERR_CUDA;
+    // A is either quantized (row_bytes per row) or, quantized in the kernel, bf16 (2 K bytes per row)
+    if (!make_map(&tb, B_q, row_bytes, args.N, 128) ||
+        !make_map(&ta, QRULE >= 0 ? args.x : A_q, QRULE >= 0 ? 2 * static_cast<uint64_t>(args.K) : row_bytes, args.M,
+                  a_rows))
+        return MXQ_ERR_CUDA;
     args.a_box_bytes = a_rows * 128;
     args.m_tiles = 1;
     args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
@@ -1244,6 +1341,45 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
         default:
             return f32 ? dispatch_bn<2, true>(A_q, B_q, a, stream, pdl_secondary)
                        : dispatch_bn<2, false>(A_q, B_q, a, stream, pdl_secondary);
+    }
+}
+
+namespace {
+template <int KIND, bool F32>
+int fused_rule(const void* W_q, const GemmArgs& a, int rule, int splits, cudaStream_t stream) {
+    return rule == MXQ_RULE_CEIL ? run_splitk<KIND, F32, MXQ_RULE_CEIL>(nullptr, W_q, a, splits, stream, true)
+                                 : run_splitk<KIND, F32, MXQ_RULE_EVEN>(nullptr, W_q, a, splits, stream, true);
+}
+}  // namespace
+
+int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
+                        int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,
+                        cudaStream_t stream) {
+    // the bf16 activations of a stage (rows rounded up to 8, BK elements) must fit the A buffer
+    if (M > 32) return kNotFused;
+    const int bk = fmt == MXQ_MXFP8 ? Cfg<2, 128, 6>::BK : Cfg<0, 128, 6>::BK;
+    const int splits = splitk_count(N, K, bk);
+    if (splits < 2) return kNotFused;
+    GemmArgs a = {};
+    a.x = x;
+    a.b_sf = W_sf;
+    a.g_a = g_A;
+    a.g_b = g_W;
+    a.out = out;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.sf_col_tiles = static_cast<int>(ceil_div(K / block_size(fmt), 4));
+    a.b_row_tiles = static_cast<int>(ceil_div(N, 128));
+    a.status = status_ptr();
+    const bool f32 = out_type == MXQ_OUT_FP32;
+    switch (fmt) {
+        case MXQ_MXFP4:
+            return f32 ? fused_rule<0, true>(W_q, a, rule, splits, stream) : fused_rule<0, false>(W_q, a, rule, splits, stream);
+        case MXQ_NVFP4:
+            return f32 ? fused_rule<1, true>(W_q, a, rule, splits, stream) : fused_rule<1, false>(W_q, a, rule, splits, stream);
+        default:
+            return f32 ? fused_rule<2, true>(W_q, a, rule, splits, stream) : fused_rule<2, false>(W_q, a, rule, splits, stream);
     }
 }
 

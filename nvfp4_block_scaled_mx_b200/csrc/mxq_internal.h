@@ -47,6 +47,15 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
                 const float* g_B, int64_t M, int64_t N, int64_t K, int fmt, int out_type, void* out,
                 cudaStream_t stream, bool pdl_secondary);
 
+// Few-token linear layer in one launch: the split-K GEMM quantizes the bf16 activations x itself
+// (rule `rule` for MX formats, global scale g_A for NVFP4) with the quantizer's arithmetic, so the
+// result equals quantize-then-GEMM bit for bit.  Returns kNotFused (nothing launched) unless the
+// problem takes the split-K kernel with M <= 32 (several K splits); arguments already validated.
+constexpr int kNotFused = 1;
+int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
+                        int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,
+                        cudaStream_t stream);
+
 // Weight-only (W4A16) GEMM launch (arguments already validated).
 int launch_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const float* g_W, int64_t M, int64_t N,
                  int64_t K, int fmt, int out_type, void* out, cudaStream_t stream);

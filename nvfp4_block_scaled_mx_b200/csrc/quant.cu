@@ -11,6 +11,7 @@
 
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
+#include "quant_block.cuh"
 
 namespace mxq {
 namespace {
@@ -44,13 +45,6 @@ __device__ __forceinline__ uint4 ld_nc(const uint4* p) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t amax_bits16(const uint32_t* w, int n) {
-    // max |bf16| over 2n values held as bf16x2 words, as an fp32 bit pattern
-    uint32_t m = w[0] & 0x7FFF7FFFu;
-    for (int i = 1; i < n; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-    return max(m & 0xFFFFu, m >> 16) << 16;
-}
-
 // Scale byte offset of block `blk` (row-major block index) in the requested layout.
 template <bool SWZ>
 __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks, uint64_t kb_magic, uint32_t col_tiles) {
@@ -60,59 +54,6 @@ __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks,
     return swz_offset(row, kc, col_tiles);
 }
 
-// One NVFP4 block of 16 elements (8 bf16x2 words): the IEEE fp32 scale sequence t = fl(amax/6),
-// u = fl(t/g), s = E4M3(u) (round to nearest even, saturating), d = fl(dec(s) * g), r = fl(1/d),
-// then the elements fl(x * r) to E2M1.  d and r come from per-code tables (nvfp4_tables); s is at
-// most 0x7E, as u is not negative and saturates to 448.  Writes 8 bytes of codes, returns s.
-template <bool OBS>
-__device__ __forceinline__ uint32_t nvfp4_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
-                                                uint32_t* codes, uint32_t& seen) {
-    const float amax = __uint_as_float(amax_bits16(wb, 8));
-    if (OBS) seen = max(seen, __float_as_uint(amax));
-    uint32_t s = 0;
-    if (amax != 0.0f) {
-        const float t = __fdiv_rn(amax, 6.0f);
-        const float uu = __fdiv_rn(t, g);
-        s = cvt_e4m3x2(uu, 0.0f) & 0xFFu;
-    }
-    const float d = tab_d[s];
-    if (d == 0.0f) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t packed = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                packed |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
-                packed |= (wb[4 * h + i] >> 31) << (8 * i + 7);
-            }
-            codes[h] = packed;
-        }
-    } else {
-        const float r = tab_r[s];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float f[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                f[2 * i] = __fmul_rn(__uint_as_float(wb[4 * h + i] << 16), r);
-                f[2 * i + 1] = __fmul_rn(__uint_as_float(wb[4 * h + i] & 0xFFFF0000u), r);
-            }
-            codes[h] = cvt_e2m1x8(f);
-        }
-    }
-    return s;
-}
-
-// d = fl(dec(s) * g) and r = fl(1/d) (0 where d is 0) for the 128 non-negative E4M3 codes s,
-// filled by the first 128 threads of a CTA.
-__device__ __forceinline__ void nvfp4_tables(float g, float* tab_d, float* tab_r) {
-    if (threadIdx.x < 128) {
-        const float d = __fmul_rn(e4m3_decode_pos(threadIdx.x), g);
-        tab_d[threadIdx.x] = d;
-        tab_r[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d)
-    }
-}
-
 // Quantize one 32-element row w (16 bf16x2 words) with unit index u: one MX block (MXFP4 / MXFP8)
 // or two NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8), coalesced across the warp.
 template <int FMT, int RULE, bool SWZ, bool OBS>
@@ -120,52 +61,22 @@ __device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u
                                               const float* tab_r, uint32_t kblocks, uint64_t kb_magic,
                                               uint32_t col_tiles, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                                               uint32_t& seen) {
-    if constexpr (FMT == MXQ_NVFP4) {
-        uint32_t codes[4];
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const uint32_t s = nvfp4_block<OBS>(w + 8 * b, g, tab_d, tab_r, codes + 2 * b, seen);
-            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
-                static_cast<uint8_t>(s);
-        }
-        reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    uint32_t codes[8];
+    const uint32_t sc = quantize32<FMT, RULE, OBS>(w, g, tab_d, tab_r, codes, seen);
+    if constexpr (FMT == MXQ_MXFP8) {
+        uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
+        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
     } else {
-        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
-        // CEIL moves one binade up when the amax mantissa exceeds elem_max's (1.5 for E2M1, 1.75 for E4M3)
-        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
-        const uint32_t abits = amax_bits16(w, 16);
-        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
-        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
-        e = max(e, -127);
-        const float inv = exp2_neg(e);
-        if constexpr (FMT == MXQ_MXFP8) {
-            uint32_t codes[8];
+        reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    }
+    if constexpr (FMT == MXQ_NVFP4) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float a0 = __fmul_rn(__uint_as_float(w[2 * i] << 16), inv);
-                const float a1 = __fmul_rn(__uint_as_float(w[2 * i] & 0xFFFF0000u), inv);
-                const float b0 = __fmul_rn(__uint_as_float(w[2 * i + 1] << 16), inv);
-                const float b1 = __fmul_rn(__uint_as_float(w[2 * i + 1] & 0xFFFF0000u), inv);
-                codes[i] = cvt_e4m3x2(a0, a1) | (cvt_e4m3x2(b0, b1) << 16);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
-            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        } else {
-            uint32_t codes[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    f[2 * i] = __fmul_rn(__uint_as_float(w[4 * h + i] << 16), inv);
-                    f[2 * i + 1] = __fmul_rn(__uint_as_float(w[4 * h + i] & 0xFFFF0000u), inv);
-                }
-                codes[h] = cvt_e2m1x8(f);
-            }
-            reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        }
-        sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(e + 127);
+        for (int b = 0; b < 2; ++b)
+            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
+                static_cast<uint8_t>(sc >> (8 * b));
+    } else {
+        sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(sc);
     }
 }
 
@@ -202,6 +113,11 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
         if (n_boxes > 0) prefetch_tmap(&tmap_x);
         for (int st = 0; st < kQuantStages; ++st) mbar_init(&full[st], 1);
         fence_barrier_init();
+    }
+    // launched with programmatic serialization: everything above overlaps the previous kernel on
+    // the stream; inputs are read and outputs written only after it has completed
+    pdl_wait();
+    if (threadIdx.x == 0) {
         const uint64_t pol = policy_evict_first();
         for (int st = 0; st < kQuantStages; ++st) {
             const int64_t b = blockIdx.x + st * step;
@@ -312,10 +228,19 @@ cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, vo
     // ceil(2^64 / kblocks); unused when kblocks == 1
     const uint64_t kb_magic =
         kblocks > 1 ? static_cast<uint64_t>(((static_cast<unsigned __int128>(1) << 64) + kblocks - 1) / kblocks) : 0;
-    kern<<<static_cast<unsigned>(blocks), kQuantBoxThreads, kQuantSmem, stream>>>(
-        tmap, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf), amax_out,
-        status_ptr(), static_cast<const uint8_t*>(x) + n_units * 64, tail);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(kQuantBoxThreads);
+    cfg.dynamicSmemBytes = kQuantSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
+                              static_cast<uint8_t*>(sf), amax_out, status_ptr(),
+                              static_cast<const void*>(static_cast<const uint8_t*>(x) + n_units * 64), tail);
 }
 
 template <int FMT, int RULE, bool SWZ>

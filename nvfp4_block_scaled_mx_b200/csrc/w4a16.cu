@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // launched with programmatic serialization: inputs are read, outputs written after this
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     const int num_tiles = p.m_tiles * p.n_tiles;
     if (warp == 0) {
@@ -553,6 +555,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     tc_fence_after();
     if constexpr (SPLIT) cluster_arrive_relaxed();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // launched with programmatic serialization: inputs are read, outputs written after this
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     // tiles: tokens fastest; a SPLIT cluster takes one tile and a contiguous range of K stages
     const int num_tiles = p.t_tiles * p.w_tiles;
@@ -951,9 +955,17 @@ int run_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w,
         attr_done[dev] = true;
     }
     const int64_t tiles = static_cast<int64_t>(args.m_tiles) * args.n_tiles;
-    const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-    kern<<<grid, kW16Threads, C::SMEM_BYTES, stream>>>(ta, tw, tsf, args);
-    return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count()));
+    cfg.blockDim = dim3(kW16Threads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, tsf, args) == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 template <int FMT, int NT, int STAGES, int AS, bool SPLIT, int DQW, bool F32>
@@ -992,15 +1004,19 @@ int run_w16t(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w
     cfg.blockDim = dim3(kWtThreads);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // programmatic serialization: the prologue may overlap the tail of the previous kernel
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if constexpr (SPLIT) {
         cfg.gridDim = dim3(static_cast<unsigned>(tiles * splits));
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(splits);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     } else {
         // 16 dequantizing warps include the epilogue warps: every CTA must own exactly one tile
         if (DQW == 16 && tiles > sm_count()) return MXQ_ERR_UNSUPPORTED;

@@ -110,7 +110,8 @@ def test_gemm_scale_placement(fmt):
 
 
 @pytest.mark.parametrize("fmt,M,N,K", [("mxfp4", 16, 256, 256), ("mxfp4", 200, 333, 640), ("nvfp4", 130, 520, 1024),
-                                       ("mxfp8", 64, 96, 512)])
+                                       ("mxfp8", 64, 96, 512), ("mxfp4", 32, 256, 1280), ("nvfp4", 64, 384, 1024),
+                                       ("mxfp8", 100, 200, 640)])
 def test_linear_matches_oracle(fmt, M, N, K):
     """mxq_linear (dynamic activation quantization + GEMM) == oracle quantize + fp64 GEMM."""
     A = synth.random_bf16((M, K), 99 + M, std=1.0)
@@ -131,6 +132,34 @@ def test_linear_matches_oracle(fmt, M, N, K):
             check_fp32(gpu, ref, abs_sum, "linear %s" % fmt)
         else:
             check_bf16(gpu, ref, abs_sum, "linear %s" % fmt)
+
+
+@pytest.mark.parametrize("fmt,rule", [("mxfp4", "ceil"), ("mxfp4", "even"), ("nvfp4", "ceil"), ("mxfp8", "ceil"),
+                                      ("mxfp8", "even")])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (32, 512, 2048), (17, 300, 320), (7, 96, 5120), (100, 300, 320),
+                                   (128, 640, 768)])
+def test_linear_one_launch_equals_quantize_then_gemm(fmt, rule, M, N, K):
+    """Up to 32 tokens: mxq_linear's GEMM quantizes the activations itself (one launch).  Its output
+    equals quantizing with mxq_quantize and multiplying with mxq_gemm, bit for bit, including a K
+    tail that leaves the last stage partly empty (K = 320), ragged and single-token problems; the
+    M = 100 and 128 cases take the two-launch path."""
+    if fmt == "mxfp8" and K % 32:
+        pytest.skip("K")
+    A = synth.random_bf16((M, K), 7 + M + K, std=1.0).cuda()
+    W = synth.random_bf16((N, K), 8 + N, std=0.02).cuda()
+    g_w = g_a = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(W)
+        g_a, _ = mxq.global_scale(A)
+    Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w)
+    Aq, Asf = mxq.quantize(A, fmt, rule, global_scale=g_a)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        two = mxq.gemm(Aq, Asf, Wq, Wsf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a, g_B=g_w)
+        one = mxq.linear(A, Wq, Wsf, N, fmt, act_rule=rule, out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+        torch.cuda.synchronize()
+        assert torch.equal(one.view(torch.int32 if out_dtype == torch.float32 else torch.int16),
+                           two.view(torch.int32 if out_dtype == torch.float32 else torch.int16)), (fmt, rule, M, N, K)
+    assert mxq.mxq_device_status(reset=True) == 0
 
 
 def test_tiny_config_full():
