@@ -344,6 +344,11 @@ def other_workloads(stream, bf16_tflops):
             tq = time_flushed(lambda: mxq.quantize_running(A, st_in, st_out, q_out=q, sf_out=sf, stream=stream), 10,
                               stream, flush)
             r["quantize_running_gbs"] = round(QUANT_BYTES_PER_ELEM["nvfp4"] * M * K / tq / 1e9, 1)
+            # the plain NVFP4 activation quantizer (static global scale) on the same tensor
+            tq = time_flushed(lambda: mxq.quantize(A, "nvfp4", global_scale=g_a, q_out=q, sf_out=sf, stream=stream), 10,
+                              stream, flush)
+            r["quantize_gbs"] = round(QUANT_BYTES_PER_ELEM["nvfp4"] * M * K / tq / 1e9, 1)
+            r["quantize_frac_of_measured_hbm"] = round(r["quantize_gbs"] / peaks()[0], 4)
             del q, sf, flush
         res[name] = r
         del A, W_q, W_sf, ws, out

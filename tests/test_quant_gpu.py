@@ -49,6 +49,30 @@ def test_quantize_matches_oracle(fmt, rule, shape):
             assert np.array_equal(sf, oracle.swizzle(sf_ref)), "swizzled scales (incl. zero padding) differ"
 
 
+@pytest.mark.parametrize("g", ["tensor", 1.0, 2.0 ** -20, 3.7e-3, 1.0e4, 2.0 ** -100, 2.0 ** 100])
+def test_nvfp4_every_block_amax(g):
+    """Every positive finite bf16 value is the amax of one 16-element NVFP4 block (its other
+    elements are seeded fractions of it, both signs), so the scale sequence t = fl(amax / 6),
+    u = fl(t / g) runs over every block amax the format can meet: scales and codes must equal the
+    oracle's IEEE fp32 arithmetic bit for bit, for the tensor's own global scale and for fixed ones
+    that send most scales to 0, saturate them at 448, or make t and u subnormal."""
+    pats = np.arange(1, 0x7F80, dtype=np.uint16)  # 0x0001 .. 0x7F7F: every positive finite bf16
+    nb, K = pats.size, 256
+    rows = (nb * 16 + K - 1) // K
+    amax = torch.from_numpy(pats.view(np.int16).copy()).view(torch.bfloat16).float()
+    frac = torch.from_numpy(np.random.default_rng(5).uniform(-1.0, 1.0, size=(nb, 16))).float()
+    frac[:, 0], frac[:, 1] = 1.0, -1.0
+    blocks = (amax[:, None] * frac).to(torch.bfloat16).reshape(-1)
+    x = torch.zeros(rows * K, dtype=torch.bfloat16)
+    x[: blocks.numel()] = blocks
+    x = x.reshape(rows, K)
+    gv = oracle.global_scale(x)[0] if g == "tensor" else float(g)
+    q_ref, sf_ref = oracle_quantize(x, "nvfp4", "even", gv)
+    q, sf = _run(x, "nvfp4", "even", mxq.SF_ROWMAJOR, float(gv))
+    assert np.array_equal(sf.reshape(sf_ref.shape), sf_ref), "scales differ (g = %r)" % (gv,)
+    assert np.array_equal(q, q_ref), "codes differ (g = %r)" % (gv,)
+
+
 @pytest.mark.parametrize("fmt,rule", COMBOS)
 def test_quantize_random_fuzz(fmt, rule):
     """Seeded fuzz over plain Gaussian data with per-row dynamic range, many blocks."""
