@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 #pragma unroll
                 for (int i = 0; i < ITEMS; ++i) {
                     const int id = t + 128 * i;
-                    const int row = id % BN, half = id / BN;
+                    const int row = id >> 1, half = id & 1;  // a warp reads 512 contiguous bytes of codes
                     codes[i] = ld_shared_v4(w_s + row * 32 + half * 16);
                     const int r_abs = nt * BN + row;
                     const int g = (r_abs >> 7) - ((nt * BN) >> 7), rr = r_abs & 127;
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 #pragma unroll
                 for (int i = 0; i < ITEMS; ++i) {
                     const int id = t + 128 * i;
-                    const int row = id % BN, half = id / BN;
+                    const int row = id >> 1, half = id & 1;  // a warp reads 512 contiguous bytes of codes
                     const uint32_t rbase = b_s + row * 128;
                     const uint32_t sw = static_cast<uint32_t>(row & 7);
                     uint4 o0, o1, o2, o3;
