@@ -587,7 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t w[UPT][16];
 #pragma unroll
                 for (int u = 0; u < UPT; ++u) {
-                    const int v = qt + u * 128, row = v / UPR, jj = v - row * UPR;
+                    // a warp takes 32 rows of one unit column (conflict-free reads); up to 8 rows, a
+                    // warp takes 4 rows x 8 unit columns (fewer units per thread)
+                    const int v = qt + u * 128;
+                    const int row = p.M > 8 ? (v & 31) : v / UPR, jj = p.M > 8 ? (v >> 5) : v % UPR;
                     if (row < p.M && static_cast<int64_t>(ks) * C::BK + jj * 32 < p.K) {
                         const uint32_t rb = a_s + (jj >> 1) * p.a_box_bytes + row * 128;
 #pragma unroll
@@ -603,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 named_barrier_sync(bar_id, 4 * 32);  // ... before any thread overwrites the buffer with codes
 #pragma unroll
                 for (int u = 0; u < UPT; ++u) {
-                    const int v = qt + u * 128, row = v / UPR, j = v - row * UPR;
+                    const int v = qt + u * 128;
+                    const int row = p.M > 8 ? (v & 31) : v / UPR, j = p.M > 8 ? (v >> 5) : v % UPR;
                     if (row >= p.M || static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
                     uint32_t codes[8], seen = 0;
                     const uint32_t sc =
