@@ -43,7 +43,9 @@ struct W16Cfg {
     static constexpr int OFF_W = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_W + STAGES * W_BYTES;
     static constexpr int OFF_B = (OFF_SF + STAGES * SF_BYTES + 1023) / 1024 * 1024;
-    static constexpr int OFF_BAR = OFF_B + BUFS * B_BYTES;
+    static constexpr int STG_BYTES = 32 * 64;  // per epilogue warp: 32 rows x 32 bf16 columns (64B swizzle)
+    static constexpr int OFF_STG = OFF_B + BUFS * B_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + kW16EpiWarps * STG_BYTES;
     static constexpr int N_BARS = 2 * STAGES + 2 * BUFS + 2;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
@@ -61,6 +63,7 @@ struct W16Args {
     int sf_col_tiles;  // ceil(K / bs / 4)
     int m_tiles, n_tiles, k_stages;
     uint32_t a_box_bytes;  // bytes of one A load (rows rounded up to 8, at most BM)
+    int tma_store;         // bf16 output through TMA stores (rows of N * 2 bytes are 16-byte multiples)
     int* status;
 };
 
@@ -149,7 +152,8 @@ __device__ __forceinline__ bool mx_scales_in_range(uint32_t codes, int n) {
 template <int FMT, int BMT, int BN, bool OUT_F32>
 __global__ void __launch_bounds__(kW16Threads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_w,
-                 const __grid_constant__ CUtensorMap tma_sf, const W16Args p) {
+                 const __grid_constant__ CUtensorMap tma_sf, const __grid_constant__ CUtensorMap tma_out,
+                 const W16Args p) {
     using C = W16Cfg<FMT, BMT, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0 && lane == 0) {
+        if (!OUT_F32 && p.tma_store) prefetch_tmap(&tma_out);
         prefetch_tmap(&tma_a);
         prefetch_tmap(&tma_w);
         prefetch_tmap(&tma_sf);
@@ -373,6 +378,46 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             tc_fence_after();
             const int m = mt * C::BM + h * 128 + sub * 32 + lane;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(h * BN + c0);
+            if (!OUT_F32 && p.tma_store) {
+                // 32 x 32 bf16 tiles through this warp's staging buffer (64B swizzle: 16-byte piece q
+                // of row r at piece q ^ ((r >> 1) & 3)) and one TMA store each, clipped at the M and N
+                // edges; the accumulator is released right after its last columns are in registers
+                uint8_t* stg = smem + C::OFF_STG + e * C::STG_BYTES;
+                const uint32_t st_row = smem_u32(stg) + lane * 64;
+                const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll 1
+                for (int c = 0; c < NC; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c, r);
+                    tmem_ld_wait();
+                    if (c + 32 == NC) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acce);
+                    }
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const __nv_bfloat162 b = __floats2bfloat162_rn(w16_epilogue<FMT>(__uint_as_float(r[2 * i]), alpha),
+                                                                       w16_epilogue<FMT>(__uint_as_float(r[2 * i + 1]), alpha));
+                        packed[i] = *reinterpret_cast<const uint32_t*>(&b);
+                    }
+                    if (lane == 0) bulk_wait_group_read0();  // the staging tile is free again
+                    __syncwarp();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(st_row + ((q ^ sw) << 4),
+                                     make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tma_out, stg, nt * BN + c0 + c, mt * C::BM + h * 128 + sub * 32);
+                        bulk_commit_group();
+                    }
+                }
+                acc_phase ^= 1u;
+                continue;
+            }
 #pragma unroll 1
             for (int c = 0; c < NC; c += 32) {
                 uint32_t r[32];
@@ -425,6 +470,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             if (lane == 0) mbar_arrive(acce);
             acc_phase ^= 1u;
         }
+        if (!OUT_F32 && p.tma_store && lane == 0) bulk_wait_group0();  // the output has left shared memory
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -870,6 +917,20 @@ bool make_a16_map(CUtensorMap* m, const void* A, int64_t M, int64_t K, uint32_t 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 out [M][N]: boxes of 32 columns (64 bytes) x 32 rows, 64B swizzle (16-byte piece q of row r
+// at piece q ^ ((r >> 1) & 3)); TMA stores clip at the M and N edges.
+bool make_out32_map(CUtensorMap* m, void* out, int64_t M, int64_t N) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // packed FP4 W [N][K/2]: boxes of 32 bytes (64 elements) x box_rows, no swizzle.
 bool make_w4_map(CUtensorMap* m, const void* W, int64_t N, int64_t K, uint32_t box_rows) {
     auto enc = encode_fn();
@@ -930,11 +991,17 @@ int run_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w,
     using C = W16Cfg<FMT, BMT, BN>;
     auto kern = w4a16_kernel<FMT, BMT, BN, F32>;
     const uint32_t a_rows = static_cast<uint32_t>(M >= C::BM ? C::BM : ceil_div(M, 8) * 8);
-    CUtensorMap ta, tw, tsf;
+    CUtensorMap ta, tw, tsf, to;
     if (!make_a16_map(&ta, A, M, K, a_rows) || !make_w4_map(&tw, Wq, N, K, BN) ||
         !make_w_sf_map(&tsf, Wsf, N, K / C::BS))
         return MXQ_ERR_CUDA;
+    const bool tma_store = !F32 && N % 8 == 0;
+    if (!tma_store)
+        to = tw;  // the output is stored directly; the map is not used
+    else if (!make_out32_map(&to, out, M, N))
+        return MXQ_ERR_CUDA;
     W16Args args = {};
+    args.tma_store = tma_store ? 1 : 0;
     args.g_w = g_w;
     args.out = out;
     args.M = static_cast<int>(M);
@@ -965,7 +1032,7 @@ int run_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float* g_w,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tw, tsf, args) == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, tsf, to, args) == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 template <int FMT, int NT, int STAGES, int AS, bool SPLIT, int DQW, bool F32>
