@@ -323,46 +323,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (!OUT_F32) {
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(m) * p.N;
                 const bool vec = (n0 + COLS <= p.N) && (p.N & 7) == 0;
-                // drain this warp's columns into registers (two TMEM loads per wait), release the
-                // accumulator, then store: the stores overlap the next tile's mainloop
-                uint32_t packed[COLS / 2];
+                // drain this warp's columns 64 at a time into registers (two TMEM loads per wait)
+                // and store them; the accumulator is released once its last columns are loaded, so
+                // the last stores overlap the next tile's mainloop
 #pragma unroll
-                for (int c = 0; c < COLS / 32; c += 2) {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld_32x32b_x32(t_row + c * 32, r0);
-                    tmem_ld_32x32b_x32(t_row + c * 32 + 32, r1);
-                    tmem_ld_wait();
+                for (int hb = 0; hb < COLS; hb += 64) {
+                    uint32_t packed[32];
+                    {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld_32x32b_x32(t_row + hb, r0);
+                        tmem_ld_32x32b_x32(t_row + hb + 32, r1);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float lo = __uint_as_float(r0[2 * i]), hi = __uint_as_float(r0[2 * i + 1]);
-                        float lo1 = __uint_as_float(r1[2 * i]), hi1 = __uint_as_float(r1[2 * i + 1]);
-                        if (KIND == 1) {
-                            lo = __fmul_rn(lo, alpha);
-                            hi = __fmul_rn(hi, alpha);
-                            lo1 = __fmul_rn(lo1, alpha);
-                            hi1 = __fmul_rn(hi1, alpha);
+                        for (int i = 0; i < 16; ++i) {
+                            float lo = __uint_as_float(r0[2 * i]), hi = __uint_as_float(r0[2 * i + 1]);
+                            float lo1 = __uint_as_float(r1[2 * i]), hi1 = __uint_as_float(r1[2 * i + 1]);
+                            if (KIND == 1) {
+                                lo = __fmul_rn(lo, alpha);
+                                hi = __fmul_rn(hi, alpha);
+                                lo1 = __fmul_rn(lo1, alpha);
+                                hi1 = __fmul_rn(hi1, alpha);
+                            }
+                            const __nv_bfloat162 b0 = __floats2bfloat162_rn(lo, hi);
+                            const __nv_bfloat162 b1 = __floats2bfloat162_rn(lo1, hi1);
+                            packed[i] = *reinterpret_cast<const uint32_t*>(&b0);
+                            packed[16 + i] = *reinterpret_cast<const uint32_t*>(&b1);
                         }
-                        const __nv_bfloat162 b0 = __floats2bfloat162_rn(lo, hi);
-                        const __nv_bfloat162 b1 = __floats2bfloat162_rn(lo1, hi1);
-                        packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&b0);
-                        packed[c * 16 + 16 + i] = *reinterpret_cast<const uint32_t*>(&b1);
                     }
-                }
-                tc_fence_before();
-                mbar_arrive(&acce[acc]);
-                if (m < p.M) {
-                    if (vec) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + n0);
+                    if (hb + 64 == COLS) {
+                        tc_fence_before();
+                        mbar_arrive(&acce[acc]);
+                    }
+                    if (m < p.M) {
+                        if (vec) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + n0 + hb);
 #pragma unroll
-                        for (int v = 0; v < COLS / 8; ++v)
-                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                    } else {
-                        uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                        } else {
+                            uint16_t* o16 = reinterpret_cast<uint16_t*>(orow);
 #pragma unroll
-                        for (int v = 0; v < COLS / 2; ++v) {
-                            const int n = n0 + 2 * v;
-                            if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
-                            if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                            for (int v = 0; v < 32; ++v) {
+                                const int n = n0 + hb + 2 * v;
+                                if (n < p.N) o16[n] = static_cast<uint16_t>(packed[v] & 0xFFFFu);
+                                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[v] >> 16);
+                            }
                         }
                     }
                 }
@@ -1314,6 +1319,9 @@ int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStre
     if (args.M > 128) return run_pair<KIND, 5, 256, F32>(A_q, B_q, args, stream, pdl);
     const int splits = splitk_count(args.N, args.K, Cfg<KIND, 128, 6>::BK);
     if (splits > 1) return run_splitk<KIND, F32>(A_q, B_q, args, splits, stream, pdl);
+    // more 128-wide tiles than SMs: 128 x 256 tiles halve the tile count (one tile per CTA up to
+    // N = 256 x SMs) and read the A rows once per 256 weight rows
+    if (ceil_div(args.N, 128) > sm_count()) return run<KIND, 256, 4, F32>(A_q, B_q, args, stream, pdl);
     return run<KIND, 128, 6, F32>(A_q, B_q, args, stream, pdl);
 }
 

@@ -35,9 +35,11 @@ def _gpu_gemm(a, w, M, N, K, fmt, out_dtype):
     return out.double().cpu().numpy() if out_dtype == torch.bfloat16 else to_np(out).astype(np.float64)
 
 
-# M <= 128 with several K stages runs the split-K cluster kernel; M > 128 the CTA-pair kernel
+# M <= 128 with several K stages runs the split-K cluster kernel; M > 128 the CTA-pair kernel; M <= 128
+# with more 128-row weight tiles than SMs the 128 x 256 one-CTA kernel (the last two shapes)
 SHAPES = [(1, 1, 64), (16, 256, 256), (128, 128, 128), (200, 300, 320), (129, 520, 1024), (300, 257, 576),
-          (64, 96, 5120), (512, 768, 192), (100, 1000, 2048), (128, 4096, 512), (1024, 96, 1024)]
+          (64, 96, 5120), (512, 768, 192), (100, 1000, 2048), (128, 4096, 512), (1024, 96, 1024),
+          (40, 19200, 256), (7, 19000, 512)]
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
