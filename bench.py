@@ -261,6 +261,18 @@ def run_mxq(args, world, rank, local):
                 "frac_of_datasheet": round(gemm_tflops / (9000.0 if fmt != "mxfp8" else 4500.0), 4),
                 "traffic": traffic_for("gemm_%s_%s" % (fmt, workload)),
                 "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
+    if M <= 128:
+        # few tokens: the GEMM streams its weights once (HBM-bound); timed with the L2 flushed
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        gemm_cold = time_flushed(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a,
+                                                  g_B=g_w, out=out, stream=stream), 20, stream, flush)
+        del flush
+        gbytes = W_q.numel() + W_sf.numel() + a_q.numel() + a_sf.numel() + out.numel() * out.element_size()
+        roofline = {"bound": "hbm", "kernel": "gemm_splitk_kernel / gemm_kernel (tcgen05 kind::%s, few tokens)" % kind,
+                    "achieved": round(gbytes / gemm_cold / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
+                    "frac": round(gbytes / gemm_cold / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
+                    "traffic": None, "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(gemm_cold * 1e3, 4),
+                    "l2": "flushed per launch (the launch latency is inside the time)"}
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
              "gbs": round(qb / quant_s / 1e9, 1), "frac": round(qb / quant_s / 1e9 / hbm_gbs, 4),
