@@ -154,6 +154,15 @@ int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const fl
 size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt);
 
 /*
+ * Kernels one mxq_linear call launches for this problem on the current device: 1 when the GEMM
+ * quantizes its own activations (up to 32 tokens with several K splits; the workspace then stays
+ * unused), 2 otherwise (quantizer, then GEMM).  The shape checks of mxq_linear come first (negative
+ * MXQ_ERR_* codes), then the device check (MXQ_ERR_DEVICE / MXQ_ERR_CUDA without a usable sm_100
+ * device).  Useful to plan CUDA-graph capture and to count launches.
+ */
+int mxq_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxq_fmt fmt);
+
+/*
  * Quantized linear layer: quantize x [M, K] bf16 per token with act_rule (MX) or global scale g_A
  * (NVFP4, device fp32[1]) into `workspace`, then out = A_q * W_q^T through mxq_gemm.
  * W_q / W_sf are the pre-quantized weights (SWIZZLED scales), g_W their NVFP4 global scale.

@@ -211,6 +211,14 @@ int mxq_gemm_w4a16(const void* A, const void* W_q, const uint8_t* W_sf, const fl
     return launch_w4a16(A, W_q, W_sf, g_W, M, N, K, fmt, out_type, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int mxq_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxq_fmt fmt) {
+    if (!valid_fmt(fmt)) return MXQ_ERR_UNSUPPORTED;
+    int rc = validate_gemm_shape(M, N, K, fmt);
+    if (rc != MXQ_OK) return rc;
+    if ((rc = check_device()) != MXQ_OK) return rc;
+    return linear_fused_splits(M, N, K, fmt) > 0 ? 1 : 2;
+}
+
 size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt) {
     if (!valid_fmt(fmt) || M < 1 || K < 1 || K % block_size(fmt) != 0) return 0;
     size_t qb = 0;

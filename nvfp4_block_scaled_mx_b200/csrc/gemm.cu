@@ -1364,13 +1364,18 @@ int fused_rule(const void* W_q, const GemmArgs& a, int rule, int splits, cudaStr
 }
 }  // namespace
 
+int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt) {
+    // the bf16 activations of a stage (rows rounded up to 8, BK elements) must fit the A buffer
+    if (M > 32) return 0;
+    const int bk = fmt == MXQ_MXFP8 ? Cfg<2, 128, 6>::BK : Cfg<0, 128, 6>::BK;
+    const int splits = splitk_count(N, K, bk);
+    return splits < 2 ? 0 : splits;
+}
+
 int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
                         int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,
                         cudaStream_t stream) {
-    // the bf16 activations of a stage (rows rounded up to 8, BK elements) must fit the A buffer
-    if (M > 32) return kNotFused;
-    const int bk = fmt == MXQ_MXFP8 ? Cfg<2, 128, 6>::BK : Cfg<0, 128, 6>::BK;
-    const int splits = splitk_count(N, K, bk);
+    const int splits = linear_fused_splits(M, N, K, fmt);
     if (splits < 2) return kNotFused;
     GemmArgs a = {};
     a.x = x;

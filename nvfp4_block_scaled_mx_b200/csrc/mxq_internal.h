@@ -52,6 +52,8 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
 // result equals quantize-then-GEMM bit for bit.  Returns kNotFused (nothing launched) unless the
 // problem takes the split-K kernel with M <= 32 (several K splits); arguments already validated.
 constexpr int kNotFused = 1;
+// K splits of the one-launch path for this problem on the current device, 0 when it does not apply.
+int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt);
 int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
                         int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,
                         cudaStream_t stream);

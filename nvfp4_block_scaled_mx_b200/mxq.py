@@ -36,6 +36,7 @@ SIGNATURES = {
     "mxq_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_gemm_w4a16": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_linear_workspace_size": (_SZ, [_I64, _I64, _I]),
+    "mxq_linear_kernel_count": (_I, [_I64, _I64, _I64, _I]),
     "mxq_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _SZ, _P, _P]),
     "mxq_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
     "mxq_device_status": (_I, [ctypes.POINTER(_I), _I, _P]),
@@ -127,6 +128,13 @@ def mxq_linear(x, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, workspa
 
 def mxq_linear_workspace_size(M, K, fmt):
     return lib().mxq_linear_workspace_size(M, K, fmt)
+
+
+def linear_kernel_count(M, N, K, fmt):
+    """Kernels one linear() call launches for this problem on the current device (1 or 2)."""
+    n = lib().mxq_linear_kernel_count(M, N, K, _fmt(fmt))
+    _check(n if n < 0 else 0, "mxq_linear_kernel_count")
+    return n
 
 
 def mxq_device_status(reset=True, stream=None):

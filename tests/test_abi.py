@@ -46,6 +46,8 @@ def test_size_helpers(L):
     ws = L.mxq_linear_workspace_size(8192, 5120, mxq.MXFP4)
     assert ws == 8192 * 2560 + 8192 * 160
     assert L.mxq_linear_workspace_size(0, 5120, mxq.MXFP4) == 0
+    assert L.mxq_linear_kernel_count(32, 5120, 96, mxq.MXFP4) == -2  # K % 64, rejected before any device check
+    assert L.mxq_linear_kernel_count(0, 5120, 5120, mxq.MXFP4) == -2
 
 
 def test_host_validation_before_launch(L):

@@ -164,6 +164,17 @@ def test_linear_one_launch_equals_quantize_then_gemm(fmt, rule, M, N, K):
     assert mxq.mxq_device_status(reset=True) == 0
 
 
+def test_linear_kernel_count():
+    """mxq_linear_kernel_count reports the one-launch path exactly where the bit-equality test above
+    exercises it: up to 32 tokens with several K splits."""
+    assert mxq.linear_kernel_count(32, 5120, 5120, "mxfp4") == 1
+    assert mxq.linear_kernel_count(1, 256, 1024, "nvfp4") == 1
+    assert mxq.linear_kernel_count(7, 96, 5120, "mxfp8") == 1
+    assert mxq.linear_kernel_count(100, 300, 320, "mxfp4") == 2
+    assert mxq.linear_kernel_count(8192, 34816, 5120, "mxfp4") == 2
+    assert mxq.linear_kernel_count(32, 34816, 5120, "mxfp4") == 2  # one K split: quantizer + GEMM
+
+
 def test_tiny_config_full():
     """The tiny MXFP4 W4A4 linear problem: every output element, fp32 out."""
     cfg = synth.CONFIGS["tiny"]
