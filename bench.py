@@ -361,6 +361,7 @@ def other_workloads(stream, bf16_tflops):
         if name == "decode":  # weight-stream bound: codes + scales of W per call
             wbytes = W_q.numel() + W_sf.numel()
             r["weight_gbs"] = round(wbytes / t / 1e9, 1)
+            r["l2"] = "back-to-back calls on one weight copy (L2-resident); --workload decode streams them from HBM"
         if name == "down_nvfp4":  # NVFP4 running-max observer quantizer on the 365 MB activation tensor
             st_in = torch.tensor([float(mxq.global_scale(A)[1].item())], dtype=torch.float32, device="cuda")
             st_out = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -396,6 +397,7 @@ def other_workloads(stream, bf16_tflops):
              "frac_of_measured_bf16": round(2.0 * M * N * K / t / 1e12 / bf16_tflops, 4)}
         if name == "decode":
             r["weight_gbs"] = round((W_q.numel() + W_sf.numel()) / t / 1e9, 1)
+            r["l2"] = "back-to-back calls on one weight copy (L2-resident)"
         res["w4a16_" + name] = r
         del A, W_q, W_sf, out
         torch.cuda.empty_cache()
