@@ -16,7 +16,6 @@
 namespace mxq {
 namespace {
 
-constexpr int kQuantThreads = 256;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     uint4 v;
@@ -37,13 +36,6 @@ __device__ __forceinline__ uint32_t div_magic(uint32_t n, uint32_t d, uint64_t m
     return d == 1 ? n : static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(n), magic));
 }
 
-// ld.global.nc with L1 allocation: the four 16-byte loads of a thread cover 64 contiguous bytes,
-// so the sector halves one load leaves in L1 serve the next.
-__device__ __forceinline__ uint4 ld_nc(const uint4* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
 
 // Scale byte offset of block `blk` (row-major block index) in the requested layout.
 template <bool SWZ>
@@ -80,6 +72,85 @@ __device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u
     }
 }
 
+__device__ __forceinline__ float e2m1_decode(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e == 0 ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
+    return (c & 8u) ? -mag : mag;
+}
+
+__device__ __forceinline__ float e4m3_decode(uint32_t c) {
+    const float mag = e4m3_decode_pos(c & 0x7Fu);
+    return (c & 0x80u) ? -mag : mag;
+}
+
+// 2^e as fp32 for e in [-127, 126] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float exp2_pos(int e) {
+    return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// One NVFP4 block of 16 elements fake-quantized: the codes and scale of nvfp4_block, decoded as
+// fl(elem * d) and rounded to bf16; 32 bytes out.
+__device__ __forceinline__ void nvfp4_fake_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
+                                                 uint4* out) {
+    uint32_t codes[2], seen = 0;
+    const uint32_t s = nvfp4_block<false>(wb, g, tab_d, tab_r, codes, seen);
+    const float d = tab_d[s];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes[h] >> (8 * i)), d), __fmul_rn(e2m1_decode(codes[h] >> (8 * i + 4)), d));
+        out[h] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// One 32-element unit fake-quantized: the codes and scales of quantize_unit, decoded in the
+// format's precision (MX: elem * 2^e, NVFP4: fl(elem * d)) and rounded once to bf16; 64 bytes out.
+template <int FMT, int RULE>
+__device__ __forceinline__ void fake_unit(const uint32_t (&w)[16], float g, const float* tab_d, const float* tab_r,
+                                          uint4* dst) {
+    if constexpr (FMT == MXQ_NVFP4) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) nvfp4_fake_block(w + 8 * b, g, tab_d, tab_r, dst + 2 * b);
+    } else {
+        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
+        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
+        const uint32_t abits = amax_bits16(w, 16);
+        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
+        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
+        e = max(e, -127);
+        const float inv = exp2_neg(e), sc = exp2_pos(e);
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+            const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+            uint32_t& oi = o[i & 3];
+            float dlo, dhi;
+            if constexpr (FMT == MXQ_MXFP8) {
+                const uint32_t c = cvt_e4m3x2(lo, hi);
+                dlo = e4m3_decode(c & 0xFFu);
+                dhi = e4m3_decode(c >> 8);
+            } else {
+                uint16_t c8;
+                asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u16.u8 %0, b;\n\t}\n"
+                    : "=h"(c8)
+                    : "f"(lo), "f"(hi));
+                dlo = e2m1_decode(c8 & 0xFu);
+                dhi = e2m1_decode(c8 >> 4);
+            }
+            oi = pack_bf16x2(__fmul_rn(dlo, sc), __fmul_rn(dhi, sc));
+            if ((i & 3) == 3) dst[i >> 2] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 constexpr int kQuantStages = 2;
 constexpr int kQuantRows = 256;                       // 64-byte rows (32 elements) per TMA box, two per thread
 constexpr int kQuantBoxThreads = kQuantRows / 2;
@@ -95,7 +166,8 @@ constexpr int kQuantSmem = kQuantStages * kQuantStageBytes + kQuantStages * 8 + 
 // with the box kQuantStages - 1 ahead.
 // OBS (NVFP4 only): gptr is a running amax; g = fl(amax / (6*448)) and the tensor amax of x is
 // folded into *amax_out with one atomicMax per warp.
-template <int FMT, int RULE, bool SWZ, bool OBS = false>
+// FAKE: fake quantization instead; q is the bf16 output (64 bytes per unit) and sf is unused.
+template <int FMT, int RULE, bool SWZ, bool OBS = false, bool FAKE = false>
 __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t n_units, uint32_t kblocks, uint64_t kb_magic,
                     uint32_t col_tiles, const float* __restrict__ gptr, uint8_t* __restrict__ q,
@@ -166,10 +238,17 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
             w1[4 * i + 3] = v1.w;
         }
         const int64_t u = b * kQuantRows + threadIdx.x;
-        if (u < n_units) quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
-        if (u + kQuantBoxThreads < n_units)
-            quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q,
-                                               sf, seen);
+        if constexpr (FAKE) {
+            uint4* y = reinterpret_cast<uint4*>(q);
+            if (u < n_units) fake_unit<FMT, RULE>(w0, g, tab_d, tab_r, y + u * 4);
+            if (u + kQuantBoxThreads < n_units) fake_unit<FMT, RULE>(w1, g, tab_d, tab_r, y + (u + kQuantBoxThreads) * 4);
+        } else {
+            if (u < n_units)
+                quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
+            if (u + kQuantBoxThreads < n_units)
+                quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, g, tab_d, tab_r, kblocks, kb_magic, col_tiles,
+                                                   q, sf, seen);
+        }
     }
     if constexpr (FMT == MXQ_NVFP4) {
         // M * K = 16 (mod 32): the last NVFP4 block is half a 32-element row, quantized from global memory
@@ -177,10 +256,15 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
             const uint4* xt = reinterpret_cast<const uint4*>(x_tail);
             const uint4 v0 = xt[0], v1 = xt[1];
             const uint32_t wt[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint32_t codes[2];
-            const uint32_t s = nvfp4_block<OBS>(wt, g, tab_d, tab_r, codes, seen);
-            reinterpret_cast<uint2*>(q)[2 * n_units] = make_uint2(codes[0], codes[1]);
-            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * n_units), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(s);
+            if constexpr (FAKE) {
+                nvfp4_fake_block(wt, g, tab_d, tab_r, reinterpret_cast<uint4*>(q) + n_units * 4);
+            } else {
+                uint32_t codes[2];
+                const uint32_t s = nvfp4_block<OBS>(wt, g, tab_d, tab_r, codes, seen);
+                reinterpret_cast<uint2*>(q)[2 * n_units] = make_uint2(codes[0], codes[1]);
+                sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * n_units), kblocks, kb_magic, col_tiles)] =
+                    static_cast<uint8_t>(s);
+            }
         }
     }
     if constexpr (OBS) {
@@ -202,7 +286,7 @@ bool make_x_map(CUtensorMap* m, const void* x, int64_t n_units) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, int RULE, bool SWZ, bool OBS>
+template <int FMT, int RULE, bool SWZ, bool OBS, bool FAKE = false>
 cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, void* q, void* sf, unsigned int* amax_out,
                          cudaStream_t stream) {
     const int64_t n_units = M * K / 32;
@@ -212,7 +296,7 @@ cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, vo
     CUtensorMap tmap;
     if (n_units > 0 && !make_x_map(&tmap, x, n_units)) return cudaErrorInvalidValue;
     if (n_units == 0) memset(&tmap, 0, sizeof(tmap));
-    auto kern = quantize_kernel<FMT, RULE, SWZ, OBS>;
+    auto kern = quantize_kernel<FMT, RULE, SWZ, OBS, FAKE>;
     int dev = 0;
     cudaGetDevice(&dev);
     static bool attr_done[64] = {};
@@ -250,122 +334,10 @@ cudaError_t launch_q(const void* x, int64_t M, int64_t K, const float* g, void* 
 
 // ------------------------------------------------------------------ fake quantization
 
-__device__ __forceinline__ float e2m1_decode(uint32_t c) {
-    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-    const float mag = e == 0 ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
-    return (c & 8u) ? -mag : mag;
-}
-
-__device__ __forceinline__ float e4m3_decode(uint32_t c) {
-    const float mag = e4m3_decode_pos(c & 0x7Fu);
-    return (c & 0x80u) ? -mag : mag;
-}
-
-// 2^e as fp32 for e in [-127, 126] (2^-127 is the subnormal 0x00400000).
-__device__ __forceinline__ float exp2_pos(int e) {
-    return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&b);
-}
-
-// One NVFP4 block of 16 elements fake-quantized: the codes and scale of nvfp4_block, decoded as
-// fl(elem * d) and rounded to bf16; 32 bytes out.
-__device__ __forceinline__ void nvfp4_fake_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
-                                                 uint4* out) {
-    uint32_t codes[2], seen = 0;
-    const uint32_t s = nvfp4_block<false>(wb, g, tab_d, tab_r, codes, seen);
-    const float d = tab_d[s];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes[h] >> (8 * i)), d), __fmul_rn(e2m1_decode(codes[h] >> (8 * i + 4)), d));
-        out[h] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-}
-
-// One thread fake-quantizes 32 consecutive elements: the same codes and scales as quantize_kernel,
-// decoded in the format's precision (MX: elem * 2^e, NVFP4: fl(elem * d)) and rounded once to bf16.
-template <int FMT, int RULE>
-__global__ void __launch_bounds__(kQuantThreads) fake_quantize_kernel(const uint4* x, int64_t n_units,
-                                                                         const float* __restrict__ gptr, uint4* y,
-                                                                         bool tail) {
-    const float g = (FMT == MXQ_NVFP4) ? *gptr : 1.0f;
-    __shared__ float tab_d[128], tab_r[128];
-    if constexpr (FMT == MXQ_NVFP4) {
-        nvfp4_tables(g, tab_d, tab_r);
-        __syncthreads();
-    }
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 v = ld_nc(x + u * 4 + i);
-            w[4 * i + 0] = v.x;
-            w[4 * i + 1] = v.y;
-            w[4 * i + 2] = v.z;
-            w[4 * i + 3] = v.w;
-        }
-        if constexpr (FMT == MXQ_NVFP4) {
-#pragma unroll
-            for (int b = 0; b < 2; ++b) nvfp4_fake_block(w + 8 * b, g, tab_d, tab_r, y + u * 4 + 2 * b);
-        } else {
-            constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
-            constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
-            const uint32_t abits = amax_bits16(w, 16);
-            int e = static_cast<int>(abits >> 23) - 127 - EMAX;
-            if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
-            e = max(e, -127);
-            const float inv = exp2_neg(e), sc = exp2_pos(e);
-            uint32_t o[4];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
-                const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
-                uint32_t& oi = o[i & 3];
-                float dlo, dhi;
-                if constexpr (FMT == MXQ_MXFP8) {
-                    const uint32_t c = cvt_e4m3x2(lo, hi);
-                    dlo = e4m3_decode(c & 0xFFu);
-                    dhi = e4m3_decode(c >> 8);
-                } else {
-                    uint16_t c8;
-                    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u16.u8 %0, b;\n\t}\n"
-                        : "=h"(c8)
-                        : "f"(lo), "f"(hi));
-                    dlo = e2m1_decode(c8 & 0xFu);
-                    dhi = e2m1_decode(c8 >> 4);
-                }
-                oi = pack_bf16x2(__fmul_rn(dlo, sc), __fmul_rn(dhi, sc));
-                if ((i & 3) == 3) y[u * 4 + (i >> 2)] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-        }
-    }
-    if constexpr (FMT == MXQ_NVFP4) {
-        // M * K = 16 (mod 32): the last block is half a 32-element unit
-        if (tail && blockIdx.x == 0 && threadIdx.x == 0) {
-            const uint4 v0 = x[n_units * 4], v1 = x[n_units * 4 + 1];
-            const uint32_t wt[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            nvfp4_fake_block(wt, g, tab_d, tab_r, y + n_units * 4);
-        }
-    }
-}
-
 template <int FMT, int RULE>
 cudaError_t launch_fq(const void* x, int64_t M, int64_t K, const float* g, void* y, cudaStream_t stream) {
-    const int64_t n_units = M * K / 32;
-    int64_t blocks = ceil_div(n_units, static_cast<int64_t>(kQuantThreads));
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    fake_quantize_kernel<FMT, RULE><<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), n_units, g, static_cast<uint4*>(y), (M * K) % 32 != 0);
-    return cudaGetLastError();
+    // the quantizer's TMA-fed ring, writing bf16 (64 bytes per 32-element unit) instead of codes
+    return launch_q_tma<FMT, RULE, false, false, true>(x, M, K, g, y, nullptr, nullptr, stream);
 }
 
 template <bool SWZ>
