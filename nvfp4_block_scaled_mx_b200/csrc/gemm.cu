@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             g_a = *p.g_a;
             const float d = __fmul_rn(e4m3_decode_pos(static_cast<uint32_t>(qt)), g_a);
             tab_d[qt] = d;
-            tab_r[qt] = d == 0.0f ? 0.0f : __frcp_rn(d);  // both groups write the same values
+            tab_r[qt] = __frcp_rn(d);  // fl(1/d), +inf for d = 0; both groups write the same values
             named_barrier_sync(bar_id, 4 * 32);
         }
         for (int ks = k0; ks < k1; ++ks) {

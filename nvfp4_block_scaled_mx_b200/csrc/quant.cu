@@ -9,6 +9,7 @@
 // directly in the swizzled tensor-core layout.
 #include <cstring>
 
+#include "dequant.cuh"
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 #include "quant_block.cuh"
@@ -72,81 +73,64 @@ __device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u
     }
 }
 
-__device__ __forceinline__ float e2m1_decode(uint32_t c) {
-    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-    const float mag = e == 0 ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
-    return (c & 8u) ? -mag : mag;
-}
-
 __device__ __forceinline__ float e4m3_decode(uint32_t c) {
     const float mag = e4m3_decode_pos(c & 0x7Fu);
     return (c & 0x80u) ? -mag : mag;
 }
 
-// 2^e as fp32 for e in [-127, 126] (2^-127 is the subnormal 0x00400000).
-__device__ __forceinline__ float exp2_pos(int e) {
-    return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&b);
-}
-
-// One NVFP4 block of 16 elements fake-quantized: the codes and scale of nvfp4_block, decoded as
-// fl(elem * d) and rounded to bf16; 32 bytes out.
-__device__ __forceinline__ void nvfp4_fake_block(const uint32_t* wb, float g, const float* tab_d, const float* tab_r,
-                                                 uint4* out) {
-    uint32_t codes[2], seen = 0;
-    const uint32_t s = nvfp4_block<false>(wb, g, tab_d, tab_r, codes, seen);
-    const float d = tab_d[s];
+// 4 E4M3 codes times an arbitrary fp32 s, rounded as fl32(elem * s) and then to bf16.
+__device__ __forceinline__ uint2 e4m3x4_fmul(uint32_t c, float s) {
+    uint32_t o[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            o[i] = pack_bf16x2(__fmul_rn(e2m1_decode(codes[h] >> (8 * i)), d), __fmul_rn(e2m1_decode(codes[h] >> (8 * i + 4)), d));
-        out[h] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 2; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(e4m3_decode((c >> (16 * i)) & 0xFFu), s),
+                                                       __fmul_rn(e4m3_decode((c >> (16 * i + 8)) & 0xFFu), s));
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
     }
+    return make_uint2(o[0], o[1]);
 }
 
-// One 32-element unit fake-quantized: the codes and scales of quantize_unit, decoded in the
-// format's precision (MX: elem * 2^e, NVFP4: fl(elem * d)) and rounded once to bf16; 64 bytes out.
+// One 32-element unit fake-quantized: the codes and scales of quantize_unit (quantize32), decoded in
+// the format's precision (MX: elem * 2^e, exact; NVFP4: fl(elem * d)) and rounded once to bf16;
+// 64 bytes out.  MX decodes multiply in bf16 by a power of two where every product is a normal
+// bf16 (scale codes [2, 128] for E2M1, [10, 134] for E4M3: exact, hence the same value), else in
+// fp32.
 template <int FMT, int RULE>
 __device__ __forceinline__ void fake_unit(const uint32_t (&w)[16], float g, const float* tab_d, const float* tab_r,
-                                          uint4* dst) {
+                                          uint4 (&dst)[4]) {
+    uint32_t codes[8], seen = 0;
+    const uint32_t sc = quantize32<FMT, RULE, false>(w, g, tab_d, tab_r, codes, seen);
     if constexpr (FMT == MXQ_NVFP4) {
+        const float d0 = tab_d[sc & 0xFFu], d1 = tab_d[sc >> 8];
+        dst[0] = dequant8_fmul(codes[0], d0);
+        dst[1] = dequant8_fmul(codes[1], d0);
+        dst[2] = dequant8_fmul(codes[2], d1);
+        dst[3] = dequant8_fmul(codes[3], d1);
+    } else if constexpr (FMT == MXQ_MXFP4) {
+        if (sc >= 2u && sc <= 128u) {
+            const uint32_t f2 = mx_factor2(sc);
 #pragma unroll
-        for (int b = 0; b < 2; ++b) nvfp4_fake_block(w + 8 * b, g, tab_d, tab_r, dst + 2 * b);
+            for (int h = 0; h < 4; ++h) dst[h] = dequant8_mul(codes[h], f2);
+        } else {
+            const float s = pow2f(static_cast<int>(sc) - 127);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) dst[h] = dequant8_cvt(codes[h], s);
+        }
     } else {
-        constexpr int EMAX = (FMT == MXQ_MXFP8) ? 8 : 2;
-        constexpr uint32_t MTHR = (FMT == MXQ_MXFP8) ? 0x600000u : 0x400000u;
-        const uint32_t abits = amax_bits16(w, 16);
-        int e = static_cast<int>(abits >> 23) - 127 - EMAX;
-        if (RULE == MXQ_RULE_CEIL) e += ((abits & 0x7FFFFFu) > MTHR) ? 1 : 0;
-        e = max(e, -127);
-        const float inv = exp2_neg(e), sc = exp2_pos(e);
-        uint32_t o[4];
+        if (sc >= 10u && sc <= 134u) {
+            const uint32_t f2 = mx8_factor2(sc);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
-            const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
-            uint32_t& oi = o[i & 3];
-            float dlo, dhi;
-            if constexpr (FMT == MXQ_MXFP8) {
-                const uint32_t c = cvt_e4m3x2(lo, hi);
-                dlo = e4m3_decode(c & 0xFFu);
-                dhi = e4m3_decode(c >> 8);
-            } else {
-                uint16_t c8;
-                asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u16.u8 %0, b;\n\t}\n"
-                    : "=h"(c8)
-                    : "f"(lo), "f"(hi));
-                dlo = e2m1_decode(c8 & 0xFu);
-                dhi = e2m1_decode(c8 >> 4);
+            for (int h = 0; h < 4; ++h) {
+                const uint2 lo = e4m3x4_mul(codes[2 * h], f2), hi = e4m3x4_mul(codes[2 * h + 1], f2);
+                dst[h] = make_uint4(lo.x, lo.y, hi.x, hi.y);
             }
-            oi = pack_bf16x2(__fmul_rn(dlo, sc), __fmul_rn(dhi, sc));
-            if ((i & 3) == 3) dst[i >> 2] = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+            const float s = pow2f(static_cast<int>(sc) - 127);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const uint2 lo = e4m3x4_fmul(codes[2 * h], s), hi = e4m3x4_fmul(codes[2 * h + 1], s);
+                dst[h] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+            }
         }
     }
 }
@@ -166,10 +150,13 @@ constexpr int kQuantSmem = kQuantStages * kQuantStageBytes + kQuantStages * 8 + 
 // with the box kQuantStages - 1 ahead.
 // OBS (NVFP4 only): gptr is a running amax; g = fl(amax / (6*448)) and the tensor amax of x is
 // folded into *amax_out with one atomicMax per warp.
-// FAKE: fake quantization instead; q is the bf16 output (64 bytes per unit) and sf is unused.
+// FAKE: fake quantization instead: each thread writes its two bf16 output rows (64 bytes per unit)
+// back over the input rows it read, and one TMA store per box (tmap_y, the same 64-byte swizzle)
+// writes the box out whole, before the slot is refilled; sf is unused.
 template <int FMT, int RULE, bool SWZ, bool OBS = false, bool FAKE = false>
 __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
-    quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t n_units, uint32_t kblocks, uint64_t kb_magic,
+    quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
+                    int64_t n_units, uint32_t kblocks, uint64_t kb_magic,
                     uint32_t col_tiles, const float* __restrict__ gptr, uint8_t* __restrict__ q,
                     uint8_t* __restrict__ sf, unsigned int* __restrict__ amax_out, int* status,
                     const void* __restrict__ x_tail, bool tail) {
@@ -183,6 +170,7 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
     const int64_t step = gridDim.x;
     if (threadIdx.x == 0) {
         if (n_boxes > 0) prefetch_tmap(&tmap_x);
+        if (FAKE && n_boxes > 0) prefetch_tmap(&tmap_y);
         for (int st = 0; st < kQuantStages; ++st) mbar_init(&full[st], 1);
         fence_barrier_init();
     }
@@ -214,6 +202,11 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
         if (__syncthreads_or(!ok)) break;
         if (threadIdx.x == 0 && it > 0) {
             const int prev = (it - 1) % kQuantStages;
+            if constexpr (FAKE) {  // the previous box's output leaves before its slot is refilled
+                tma_store_2d(&tmap_y, ring + prev * kQuantStageBytes, 0, static_cast<int>((b - step) * kQuantRows));
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            }
             const int64_t nb = b + (kQuantStages - 1) * step;
             if (nb < n_boxes) {
                 mbar_arrive_expect_tx(&full[prev], kQuantStageBytes);
@@ -239,15 +232,33 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
         }
         const int64_t u = b * kQuantRows + threadIdx.x;
         if constexpr (FAKE) {
-            uint4* y = reinterpret_cast<uint4*>(q);
-            if (u < n_units) fake_unit<FMT, RULE>(w0, g, tab_d, tab_r, y + u * 4);
-            if (u + kQuantBoxThreads < n_units) fake_unit<FMT, RULE>(w1, g, tab_d, tab_r, y + (u + kQuantBoxThreads) * 4);
+            uint4 o0[4], o1[4];
+            fake_unit<FMT, RULE>(w0, g, tab_d, tab_r, o0);
+            fake_unit<FMT, RULE>(w1, g, tab_d, tab_r, o1);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t piece = (static_cast<uint32_t>(i) ^ sw) << 4;
+                st_shared_v4(row + piece, o0[i]);
+                st_shared_v4(row + kQuantBoxThreads * 64 + piece, o1[i]);
+            }
+            fence_proxy_async_smem();  // read next by the TMA store
         } else {
             if (u < n_units)
                 quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
             if (u + kQuantBoxThreads < n_units)
                 quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, g, tab_d, tab_r, kblocks, kb_magic, col_tiles,
                                                    q, sf, seen);
+        }
+    }
+    if constexpr (FAKE) {
+        // the last box this CTA wrote (also after a timed-out wait, which ends the loop before the
+        // store at the top of the next iteration)
+        __syncthreads();
+        if (threadIdx.x == 0 && it > 0) {
+            tma_store_2d(&tmap_y, ring + ((it - 1) % kQuantStages) * kQuantStageBytes, 0,
+                         static_cast<int>((blockIdx.x + static_cast<int64_t>(it - 1) * step) * kQuantRows));
+            bulk_commit_group();
+            bulk_wait_group0();
         }
     }
     if constexpr (FMT == MXQ_NVFP4) {
@@ -257,7 +268,11 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
             const uint4 v0 = xt[0], v1 = xt[1];
             const uint32_t wt[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             if constexpr (FAKE) {
-                nvfp4_fake_block(wt, g, tab_d, tab_r, reinterpret_cast<uint4*>(q) + n_units * 4);
+                uint32_t codes[2];
+                const uint32_t s = nvfp4_block<false>(wt, g, tab_d, tab_r, codes, seen);
+                uint4* yt = reinterpret_cast<uint4*>(q) + n_units * 4;
+                yt[0] = dequant8_fmul(codes[0], tab_d[s]);
+                yt[1] = dequant8_fmul(codes[1], tab_d[s]);
             } else {
                 uint32_t codes[2];
                 const uint32_t s = nvfp4_block<OBS>(wt, g, tab_d, tab_r, codes, seen);
@@ -293,9 +308,12 @@ cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, vo
     const bool tail = (M * K) % 32 != 0;  // NVFP4 only: a last block of 16 elements
     const uint32_t kblocks = static_cast<uint32_t>(K / block_size(FMT));
     const uint32_t col_tiles = static_cast<uint32_t>(ceil_div(kblocks, 4));
-    CUtensorMap tmap;
+    CUtensorMap tmap, tmap_y;
+    memset(&tmap, 0, sizeof(tmap));
+    memset(&tmap_y, 0, sizeof(tmap_y));
     if (n_units > 0 && !make_x_map(&tmap, x, n_units)) return cudaErrorInvalidValue;
-    if (n_units == 0) memset(&tmap, 0, sizeof(tmap));
+    // fake quantization: the bf16 output has the input's layout, written box by box with TMA stores
+    if (FAKE && n_units > 0 && !make_x_map(&tmap_y, q, n_units)) return cudaErrorInvalidValue;
     auto kern = quantize_kernel<FMT, RULE, SWZ, OBS, FAKE>;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -322,7 +340,7 @@ cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, vo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmap, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
+    return cudaLaunchKernelEx(&cfg, kern, tmap, tmap_y, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
                               static_cast<uint8_t*>(sf), amax_out, status_ptr(),
                               static_cast<const void*>(static_cast<const uint8_t*>(x) + n_units * 64), tail);
 }

@@ -30,20 +30,24 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint32_t* wb, float g, con
         const float uu = __fdiv_rn(t, g);
         s = cvt_e4m3x2(uu, 0.0f) & 0xFFu;
     }
-    const float d = tab_d[s];
-    if (d == 0.0f) {
+    const float r = tab_r[s];
+    if (r == __int_as_float(0x7F800000)) {
+        // r = fl(1/d) is +inf for d = 0 (every code a signed zero) and where 1/d overflows (d below
+        // 2^-128, a subnormal g): x * r is then +-inf for x != 0, saturating to +-6, and a zero
+        // element stays a signed zero
+        const uint32_t big = tab_d[s] == 0.0f ? 0u : 7u;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t packed = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                packed |= (wb[4 * h + i] >> 15 & 1u) << (8 * i + 3);
-                packed |= (wb[4 * h + i] >> 31) << (8 * i + 7);
+                const uint32_t v = wb[4 * h + i];
+                packed |= ((v >> 15 & 1u) << 3 | ((v & 0x7FFFu) != 0 ? big : 0u)) << (8 * i);
+                packed |= ((v >> 31) << 3 | ((v & 0x7FFF0000u) != 0 ? big : 0u)) << (8 * i + 4);
             }
             codes[h] = packed;
         }
     } else {
-        const float r = tab_r[s];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             float f[8];
@@ -58,13 +62,13 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint32_t* wb, float g, con
     return s;
 }
 
-// d = fl(dec(s) * g) and r = fl(1/d) (0 where d is 0) for the 128 non-negative E4M3 codes s,
+// d = fl(dec(s) * g) and r = fl(1/d) (+inf where d is 0) for the 128 non-negative E4M3 codes s,
 // filled by the first 128 threads of a CTA.
 __device__ __forceinline__ void nvfp4_tables(float g, float* tab_d, float* tab_r) {
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(e4m3_decode_pos(threadIdx.x), g);
         tab_d[threadIdx.x] = d;
-        tab_r[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d)
+        tab_r[threadIdx.x] = __frcp_rn(d);  // correctly rounded 1/d, as fl(1/d); +inf for d = 0
     }
 }
 

@@ -173,7 +173,10 @@ static void nvfp4_block(const uint16_t* x, float g, uint8_t* codes, uint8_t* sca
             codes[i] = signbit(xv) ? 0x8u : 0x0u;
         } else {
             volatile float r = 1.0f / d;
-            volatile float v = (float)xv * r;
+            /* r overflows to +inf when d < 2^-128 (a subnormal g): x * r is then +-inf for x != 0
+             * (saturating to +-6) and NaN for x = 0, which has no E2M1 code; a zero element
+             * encodes as a zero with its sign, whatever the scale. */
+            volatile float v = xv == 0.0 ? (float)xv : (float)xv * r;
             codes[i] = orc_e2m1_encode((double)v);
         }
     }

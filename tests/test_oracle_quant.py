@@ -221,6 +221,28 @@ def test_nvfp4_hand_block(orc):
     assert np.allclose(d[0, :4], vals[:4], rtol=0, atol=0)
 
 
+def test_nvfp4_reciprocal_overflow(orc):
+    # g = 2^-140 is an fp32 subnormal.  A block with amax 1 has u = fl(fl(1/6) / g), far above 448,
+    # so s saturates to 448 (0x7E) and d = 448 * 2^-140 = 1.75 * 2^-132, whose reciprocal overflows
+    # fp32: r = +inf.  Then fl(x * r) is +-inf for every nonzero x (E2M1 saturates it to +-6, code 7
+    # with the sign) and NaN for x = +-0, which encodes as a zero with x's sign.
+    g = 2.0 ** -140
+    d = np.float32(448.0) * np.float32(g)
+    assert d == np.float32(1.75 * 2.0 ** -132)
+    with np.errstate(over="ignore", divide="ignore"):
+        assert np.isinf(np.float32(1.0) / d)
+    tiny = float(torch.tensor(2.0 ** -133, dtype=torch.bfloat16))  # the smallest bf16 subnormal
+    vals = [1.0, -1.0, 0.0, -0.0, tiny, -tiny, 0.5, -3.0] * 2
+    x = torch.tensor([vals], dtype=torch.bfloat16)
+    q, sf = orc.quantize(x, orc.NVFP4, 0, g=g)
+    assert sf[0, 0] == 0x7E
+    expect = [0x7, 0xF, 0x0, 0x8, 0x7, 0xF, 0x7, 0xF] * 2
+    assert _unpack_fp4(q)[0].tolist() == expect
+    # with g = 1/2688 the same block has d = 1/6 and r = 6: the tiny elements round to signed zeros
+    q2, _ = orc.quantize(x, orc.NVFP4, 0, g=1.0 / 2688)
+    assert _unpack_fp4(q2)[0, :6].tolist() == [0x7, 0xF, 0x0, 0x8, 0x0, 0x8]
+
+
 def test_swizzle_layout(orc):
     for rows, kb in [(1, 1), (128, 4), (130, 5), (300, 160), (16, 8)]:
         total = orc.swizzled_bytes(rows, kb)

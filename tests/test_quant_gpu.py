@@ -49,13 +49,15 @@ def test_quantize_matches_oracle(fmt, rule, shape):
             assert np.array_equal(sf, oracle.swizzle(sf_ref)), "swizzled scales (incl. zero padding) differ"
 
 
-@pytest.mark.parametrize("g", ["tensor", 1.0, 2.0 ** -20, 3.7e-3, 1.0e4, 2.0 ** -100, 2.0 ** 100])
+@pytest.mark.parametrize("g", ["tensor", 1.0, 2.0 ** -20, 3.7e-3, 1.0e4, 2.0 ** -100, 2.0 ** 100, 2.0 ** -140,
+                               1.0e-40])
 def test_nvfp4_every_block_amax(g):
     """Every positive finite bf16 value is the amax of one 16-element NVFP4 block (its other
     elements are seeded fractions of it, both signs), so the scale sequence t = fl(amax / 6),
     u = fl(t / g) runs over every block amax the format can meet: scales and codes must equal the
     oracle's IEEE fp32 arithmetic bit for bit, for the tensor's own global scale and for fixed ones
-    that send most scales to 0, saturate them at 448, or make t and u subnormal."""
+    that send most scales to 0, saturate them at 448, make t and u subnormal, or make g subnormal
+    (where fl(1/d) overflows to +inf for the large scales)."""
     pats = np.arange(1, 0x7F80, dtype=np.uint16)  # 0x0001 .. 0x7F7F: every positive finite bf16
     nb, K = pats.size, 256
     rows = (nb * 16 + K - 1) // K
