@@ -55,10 +55,14 @@ def parse():
     ap.add_argument("--no-others", action="store_true", help="skip the informational other-problem timings")
     ap.add_argument("--M", type=int, default=None, help="override the workload's M (profiling runs)")
     ap.add_argument("--N", type=int, default=None, help="override the workload's N (profiling runs)")
-    ap.add_argument("--op", default="linear", choices=["linear", "w4a16"],
-                    help="w4a16: time only the weight-only GEMM on the workload's shape (profiling runs; "
-                         "prints its own JSON line, not the benchmark line)")
-    ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4"], help="weight format of --op w4a16")
+    ap.add_argument("--op", default="linear", choices=["linear", "w4a16", "quantize", "fake_quantize"],
+                    help="time one kernel alone on the workload's shape and print its own JSON line, not the "
+                         "benchmark line (profiling runs): w4a16 = the weight-only GEMM; quantize / "
+                         "fake_quantize = the activation quantizer / fake quantizer on A [M, K]")
+    ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4", "mxfp8"],
+                    help="format of --op w4a16 (weights; mxfp4 or nvfp4), quantize and fake_quantize")
+    ap.add_argument("--rule", default="ceil", choices=["even", "ceil"], help="MX scale rule of --op quantize / "
+                    "fake_quantize")
     return ap.parse_args()
 
 
@@ -549,6 +553,8 @@ def run_w4a16_op(args):
     from nvfp4_block_scaled_mx_b200 import mxq
     if not torch.cuda.is_available():
         raise SystemExit("bench.py --op w4a16 needs a CUDA device (there is no CPU fallback)")
+    if args.fmt not in ("mxfp4", "nvfp4"):
+        raise SystemExit("bench.py --op w4a16 takes --fmt mxfp4 or nvfp4 (4-bit weights)")
     cfg = synth.CONFIGS[args.workload]
     M, N, K = args.M or cfg["M"], args.N or cfg["N"], cfg["K"]
     A = synth.random_bf16((M, K), 71, device="cuda")
@@ -571,10 +577,43 @@ def run_w4a16_op(args):
             "weight_gbs_l2_flushed": round(wbytes / cold / 1e9, 1)}
 
 
+def run_quantize_op(args):
+    """The activation quantizer (or fake quantizer) alone on A [M, K] of the workload (N(0,1) bf16),
+    timed with the L2 flushed before each launch, against the measured HBM bandwidth."""
+    from nvfp4_block_scaled_mx_b200 import mxq
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --op %s needs a CUDA device (there is no CPU fallback)" % args.op)
+    cfg = synth.CONFIGS[args.workload]
+    M, K = args.M or cfg["M"], cfg["K"]
+    A = synth.random_bf16((M, K), 73, device="cuda")
+    g = mxq.global_scale(A)[0] if args.fmt == "nvfp4" else None
+    rule = "even" if args.fmt == "nvfp4" else args.rule
+    stream = torch.cuda.current_stream()
+    if args.op == "quantize":
+        q, sf = mxq.quantize(A, args.fmt, rule, global_scale=g, stream=stream)
+        f = lambda: mxq.quantize(A, args.fmt, rule, global_scale=g, q_out=q, sf_out=sf, stream=stream)
+        bpe = QUANT_BYTES_PER_ELEM[args.fmt]
+    else:
+        y = torch.empty_like(A)
+        f = lambda: mxq.fake_quantize(A, args.fmt, rule, global_scale=g, out=y, stream=stream)
+        bpe = 4.0
+    for _ in range(max(3, args.warmup)):
+        f()
+    flush = l2_flush_buffer("cuda")
+    t = time_flushed(f, max(3, args.steps), stream, flush)
+    hbm = peaks()[0]
+    return {"op": args.op, "M": M, "K": K, "fmt": args.fmt, "rule": rule, "ms": round(t * 1e3, 4),
+            "gbs": round(bpe * M * K / t / 1e9, 1), "frac_of_measured_hbm": round(bpe * M * K / t / 1e9 / hbm, 4),
+            "algorithmic_bytes_per_elem": bpe, "l2": "flushed per launch"}
+
+
 def main():
     args = parse()
     if args.op == "w4a16":
         print(json.dumps(run_w4a16_op(args)), flush=True)
+        return
+    if args.op in ("quantize", "fake_quantize"):
+        print(json.dumps(run_quantize_op(args)), flush=True)
         return
     world, rank, local = dist_init()
     try:

@@ -48,28 +48,50 @@ __device__ __forceinline__ uint32_t scale_offset(uint32_t blk, uint32_t kblocks,
 }
 
 // Quantize one 32-element row w (16 bf16x2 words) with unit index u: one MX block (MXFP4 / MXFP8)
-// or two NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8), coalesced across the warp.
+// or two NVFP4 blocks.  Codes: 16 bytes (FP4) or 32 bytes (FP8), coalesced across the warp.  Every
+// lane of the warp calls this (rows past the end hold the TMA's zero fill; `valid` masks their
+// stores), so that the scale bytes can be gathered across lanes: when a row's block count is a
+// multiple of 4 (pack_sf), the 4 scale bytes of 4 consecutive blocks sit in one aligned 32-bit word
+// of either layout, and lane 4j (MX) or 2j (NVFP4, two blocks per unit) stores that word for
+// itself and its neighbours; otherwise each block's byte is stored on its own.
 template <int FMT, int RULE, bool SWZ, bool OBS>
-__device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u, float g, const float* tab_d,
-                                              const float* tab_r, uint32_t kblocks, uint64_t kb_magic,
-                                              uint32_t col_tiles, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-                                              uint32_t& seen) {
+__device__ __forceinline__ void quantize_unit(const uint32_t (&w)[16], int64_t u, bool valid, bool pack_sf, float g,
+                                              const float* tab_d, const float* tab_r, uint32_t kblocks,
+                                              uint64_t kb_magic, uint32_t col_tiles, uint8_t* __restrict__ q,
+                                              uint8_t* __restrict__ sf, uint32_t& seen) {
     uint32_t codes[8];
     const uint32_t sc = quantize32<FMT, RULE, OBS>(w, g, tab_d, tab_r, codes, seen);
-    if constexpr (FMT == MXQ_MXFP8) {
-        uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
-        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-    } else {
-        reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    if (valid) {
+        if constexpr (FMT == MXQ_MXFP8) {
+            uint4* dst = reinterpret_cast<uint4*>(q) + 2 * u;
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        } else {
+            reinterpret_cast<uint4*>(q)[u] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        }
     }
-    if constexpr (FMT == MXQ_NVFP4) {
+    constexpr int BLOCKS = (FMT == MXQ_NVFP4) ? 2 : 1;  // scale bytes per unit
+    const uint32_t blk = static_cast<uint32_t>(BLOCKS * u);
+    if (pack_sf) {
+        const uint32_t lane = threadIdx.x & 31u;
+        uint32_t word;
+        bool leader;
+        if constexpr (BLOCKS == 2) {
+            word = (sc & 0xFFFFu) | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 16);
+            leader = (lane & 1u) == 0;
+        } else {
+            word = (sc & 0xFFu) | ((__shfl_down_sync(0xFFFFFFFFu, sc, 1) & 0xFFu) << 8) |
+                   ((__shfl_down_sync(0xFFFFFFFFu, sc, 2) & 0xFFu) << 16) | (__shfl_down_sync(0xFFFFFFFFu, sc, 3) << 24);
+            leader = (lane & 3u) == 0;
+        }
+        // a leader's block index is a multiple of 4 and n_units * BLOCKS is too, so the word's
+        // other blocks are valid whenever the leader's is
+        if (leader && valid)
+            *reinterpret_cast<uint32_t*>(sf + scale_offset<SWZ>(blk, kblocks, kb_magic, col_tiles)) = word;
+    } else if (valid) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b)
-            sf[scale_offset<SWZ>(static_cast<uint32_t>(2 * u + b), kblocks, kb_magic, col_tiles)] =
-                static_cast<uint8_t>(sc >> (8 * b));
-    } else {
-        sf[scale_offset<SWZ>(static_cast<uint32_t>(u), kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(sc);
+        for (int b = 0; b < BLOCKS; ++b)
+            sf[scale_offset<SWZ>(blk + b, kblocks, kb_magic, col_tiles)] = static_cast<uint8_t>(sc >> (8 * b));
     }
 }
 
@@ -190,6 +212,7 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
     if constexpr (FMT == MXQ_NVFP4) nvfp4_tables(g, tab_d, tab_r);
     __syncthreads();
     uint32_t seen = 0;  // largest block amax (fp32 bits) this thread quantized, for OBS
+    const bool pack_sf = (kblocks & 3u) == 0;
     // 64-byte swizzle: 16-byte piece c of row r sits at piece c ^ ((r >> 1) & 3); this thread takes
     // rows t and t + 128 of each box, which share the same swizzle
     const uint32_t my_row = smem_u32(ring) + threadIdx.x * 64u;
@@ -243,11 +266,10 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
             }
             fence_proxy_async_smem();  // read next by the TMA store
         } else {
-            if (u < n_units)
-                quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, g, tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
-            if (u + kQuantBoxThreads < n_units)
-                quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, g, tab_d, tab_r, kblocks, kb_magic, col_tiles,
-                                                   q, sf, seen);
+            quantize_unit<FMT, RULE, SWZ, OBS>(w0, u, u < n_units, pack_sf, g, tab_d, tab_r, kblocks, kb_magic,
+                                               col_tiles, q, sf, seen);
+            quantize_unit<FMT, RULE, SWZ, OBS>(w1, u + kQuantBoxThreads, u + kQuantBoxThreads < n_units, pack_sf, g,
+                                               tab_d, tab_r, kblocks, kb_magic, col_tiles, q, sf, seen);
         }
     }
     if constexpr (FAKE) {

@@ -25,12 +25,13 @@ def _run(x_cpu, fmt, rule, layout, g=None):
 
 
 @pytest.mark.parametrize("fmt,rule", COMBOS)
-@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (5, 80), (1, 32), (3, 64), (37, 320), (130, 1056), (256, 5120),
-                                   (2053, 8192)])
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (5, 80), (1, 32), (3, 64), (7, 128), (9, 384), (37, 320),
+                                   (130, 1056), (256, 5120), (2053, 8192)])
 def test_quantize_matches_oracle(fmt, rule, shape):
     """Shapes cover a single block, NVFP4 tensors whose last 16-element block is half a 32-element
-    row of the input stream (M * K = 16 mod 32), partial 256-row input boxes, and more boxes than
-    CTAs (the input ring wraps)."""
+    row of the input stream (M * K = 16 mod 32), partial 256-row input boxes, more boxes than CTAs
+    (the input ring wraps), and rows whose block count is and is not a multiple of 4 (scale bytes
+    gathered across lanes into 32-bit stores, or stored one by one)."""
     M, K = shape
     bs = 16 if fmt == "nvfp4" else 32
     if K % bs:
