@@ -55,10 +55,12 @@ def parse():
     ap.add_argument("--no-others", action="store_true", help="skip the informational other-problem timings")
     ap.add_argument("--M", type=int, default=None, help="override the workload's M (profiling runs)")
     ap.add_argument("--N", type=int, default=None, help="override the workload's N (profiling runs)")
-    ap.add_argument("--op", default="linear", choices=["linear", "w4a16", "quantize", "fake_quantize"],
+    ap.add_argument("--op", default="linear",
+                    choices=["linear", "w4a16", "quantize", "fake_quantize", "scaled_mm"],
                     help="time one kernel alone on the workload's shape and print its own JSON line, not the "
                          "benchmark line (profiling runs): w4a16 = the weight-only GEMM; quantize / "
-                         "fake_quantize = the activation quantizer / fake quantizer on A [M, K]")
+                         "fake_quantize = the activation quantizer / fake quantizer on A [M, K]; scaled_mm = "
+                         "the block-scaled GEMM beside torch's cuBLASLt scaled_mm on the same bytes (context)")
     ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4", "mxfp8"],
                     help="format of --op w4a16 (weights; mxfp4 or nvfp4), quantize and fake_quantize")
     ap.add_argument("--rule", default="ceil", choices=["even", "ceil"], help="MX scale rule of --op quantize / "
@@ -607,8 +609,56 @@ def run_quantize_op(args):
             "algorithmic_bytes_per_elem": bpe, "l2": "flushed per launch"}
 
 
+def run_scaled_mm_op(args):
+    """Context, not a product path: the workload's block-scaled GEMM (activations and weights quantized
+    by this library) timed beside torch.nn.functional.scaled_mm, which runs cuBLASLt's block-scaled
+    GEMM on the same code and swizzled-scale bytes.  Back-to-back launches, CUDA events.  Also the
+    largest difference of the two outputs relative to the largest output (0 when they agree bit for
+    bit; NVFP4 differs by where the global scales are applied)."""
+    import torch.nn.functional as F
+    from nvfp4_block_scaled_mx_b200 import mxq
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --op scaled_mm needs a CUDA device")
+    cfg = synth.CONFIGS[args.workload]
+    M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
+    A, W = synth.make_inputs(args.workload, device="cuda")
+    g_a = g_w = None
+    if fmt == "nvfp4":
+        g_w, g_a = mxq.global_scale(W)[0], mxq.global_scale(A)[0]
+    Aq, Asf = mxq.quantize(A, fmt, cfg["a_rule"], global_scale=g_a)
+    Wq, Wsf = mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w)
+    del A, W
+    stream = torch.cuda.current_stream()
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ours = lambda: mxq.gemm(Aq, Asf, Wq, Wsf, M, N, K, fmt, g_A=g_a, g_B=g_w, out=out, stream=stream)
+    elem = torch.float8_e4m3fn if fmt == "mxfp8" else torch.float4_e2m1fn_x2
+    sdt = torch.float8_e4m3fn if fmt == "nvfp4" else torch.float8_e8m0fnu
+    rec = F.ScalingType.BlockWise1x16 if fmt == "nvfp4" else F.ScalingType.BlockWise1x32
+    sw = F.SwizzleType.SWIZZLE_32_4_4
+    lib = lambda: F.scaled_mm(Aq.view(elem), Wq.view(elem).t(), Asf.view(sdt), rec, Wsf.view(sdt), rec,
+                              swizzle_a=sw, swizzle_b=sw, output_dtype=torch.bfloat16)
+    for _ in range(max(3, args.warmup)):
+        ours()
+    t_ours = time_loop(ours, args.steps, stream)
+    ref = lib()
+    for _ in range(max(3, args.warmup)):
+        lib()
+    t_lib = time_loop(lib, args.steps, stream)
+    ours()
+    torch.cuda.synchronize()
+    r = ref.float() * (g_a * g_w) if fmt == "nvfp4" else ref.float()
+    flops = 2.0 * M * N * K
+    return {"op": "scaled_mm", "workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt,
+            "mxq_ms": round(t_ours * 1e3, 4), "mxq_tflops": round(flops / t_ours / 1e12, 1),
+            "scaled_mm_ms": round(t_lib * 1e3, 4), "scaled_mm_tflops": round(flops / t_lib / 1e12, 1),
+            "max_rel_diff": float((out.float() - r).abs().max() / r.abs().max())}
+
+
 def main():
     args = parse()
+    if args.op == "scaled_mm":
+        print(json.dumps(run_scaled_mm_op(args)), flush=True)
+        return
     if args.op == "w4a16":
         print(json.dumps(run_w4a16_op(args)), flush=True)
         return
