@@ -19,6 +19,8 @@
  * NVFP4 (fp32 IEEE, g = global scale in the decode direction, x ~ q * s * g):
  *   s = RNE_E4M3_satfinite(fl(fl(amax/6) / g)) (0 for an all-zero block), d = fl(dec(s) * g),
  *   q_i = RNE_E2M1_sat(fl(x_i * fl(1/d))); when d == 0 every code is a zero that keeps x_i's sign.
+ *   Where fl(1/d) overflows to +inf (d < 2^-128, only with an fp32-subnormal g), a nonzero x_i
+ *   saturates to +-6 and a zero x_i stays a zero with its sign (0 * inf has no E2M1 code).
  *
  * Conventions for every call:
  *   - Pointers marked (device) are device memory of the current CUDA device; the caller owns and

@@ -2,11 +2,13 @@
 // NVFP4 global scale, and the bounded-wait self-test kernel.
 //
 // The quantizer is a single streaming pass over x.  x is read as rows of 64 bytes (32 elements:
-// one MX block or two NVFP4 blocks) by TMA, 256 rows per box, into a 4-stage shared-memory ring
-// with a 64-byte swizzle; each thread then owns one 32-element row (its four 16-byte pieces sit in
-// different banks), takes the block amax on the bf16 bit patterns, derives the scale, and writes 16
-// (FP4) or 32 (FP8) bytes of packed codes plus one scale byte per block, either row-major or
-// directly in the swizzled tensor-core layout.
+// one MX block or two NVFP4 blocks) by TMA, 256 rows per box, into a 2-stage shared-memory ring
+// with a 64-byte swizzle (5 CTAs per SM); each thread then owns two 32-element rows of a box (their
+// four 16-byte pieces sit in different banks), takes the block amax on the bf16 bit patterns,
+// derives the scale, and writes 16 (FP4) or 32 (FP8) bytes of packed codes per row plus the scale
+// bytes, either row-major or directly in the swizzled tensor-core layout (4 blocks' bytes gathered
+// across lanes into one 32-bit store where a row's block count allows).  Fake quantization runs the
+// same ring and decodes the codes back to bf16 in place.
 #include <cstring>
 
 #include "dequant.cuh"
