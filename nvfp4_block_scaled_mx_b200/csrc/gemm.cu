@@ -1,6 +1,13 @@
 // gemm.cu -- block-scaled GEMM on the sm_100a tensor cores (tcgen05), out = alpha * dq(A) dq(B)^T.
 //
-// One persistent CTA per SM, warp-specialised:
+// Three kernels share the MMA, scale and epilogue plumbing, chosen on the host by shape:
+//   gemm_pair_kernel    M > 128: two-CTA clusters computing 256 x BN tiles (cta_group::2);
+//   gemm_splitk_kernel  M <= 128 with too few output tiles for the SMs: K split over a cluster,
+//                       partials reduced through distributed shared memory (and, for up to 32
+//                       rows, the activations quantized inside the kernel);
+//   gemm_kernel         M <= 128 otherwise, described here.
+//
+// gemm_kernel: one persistent CTA per SM, warp-specialised:
 //   warp 0       TMA producer: A and B tiles (128-byte K slices, 128B-swizzled) and their
 //                swizzled scale tiles (bulk copies) into a STAGES-deep shared-memory ring;
 //   warp 1       TMEM owner and MMA issuer: 4 block-scaled MMAs per stage into an fp32
