@@ -31,19 +31,20 @@ __device__ __forceinline__ uint4 dequant8_cvt(uint32_t w, float scale) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// The same on the integer and FMA pipes.  Codes 2i and 2i+1 of the word are moved to bits 0-3 and
-// 16-19 of one register (byte permute; selector nibbles 8-B yield zero bytes, as the selected bytes
-// have a clear top bit), one integer multiply by 2^6 + 2^12 copies each code to bits 6-9 and 12-15
-// (no carries: the copies do not overlap), and a mask keeps the magnitude bits at 6-8 and the sign
-// at bit 15.  That bf16 pattern s<<15 | m<<6 reads as the code's value times 2^-126 (0.5 is the
-// subnormal 0x0040), so a bf16x2 multiply by f2 = (2^126 s, 2^126 s) yields the scaled elements,
-// exactly whenever every product is a normal bf16.
+// Byte permute: result byte i is byte sel_i of the 8-byte pair {b, a} (a is bytes 0-3).
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
 }
 
+// dequant8_cvt on the integer and FMA pipes.  Codes 2i and 2i+1 of the word are moved to bits 0-3 and
+// 16-19 of one register (byte permute; selector nibbles 8-B yield zero bytes, as the selected bytes
+// have a clear top bit), one integer multiply by 2^6 + 2^12 copies each code to bits 6-9 and 12-15
+// (no carries: the copies do not overlap), and a mask keeps the magnitude bits at 6-8 and the sign
+// at bit 15.  That bf16 pattern s<<15 | m<<6 reads as the code's value times 2^-126 (0.5 is the
+// subnormal 0x0040), so a bf16x2 multiply by f2 = (2^126 s, 2^126 s) yields the scaled elements,
+// exactly whenever every product is a normal bf16.
 __device__ __forceinline__ uint4 dequant8_mul(uint32_t w, uint32_t f2) {
     const uint32_t ev = w & 0x0F0F0F0Fu;         // codes 0, 2, 4, 6 in the low nibbles of bytes 0-3
     const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
