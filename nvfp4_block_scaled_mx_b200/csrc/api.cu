@@ -44,8 +44,11 @@ int check_device() {
     return v == 1 ? MXQ_OK : MXQ_ERR_DEVICE;
 }
 
+// A dimension the library accepts: 1 <= v < 2^31 (products of two fit in 62 bits).
+bool dim_ok(int64_t v) { return v >= 1 && v < (int64_t(1) << 31); }
+
 int q_bytes(int64_t rows, int64_t K, int fmt, size_t* out) {
-    if (rows < 1 || K < 1) return MXQ_ERR_SHAPE;
+    if (!dim_ok(rows) || !dim_ok(K)) return MXQ_ERR_SHAPE;
     *out = static_cast<size_t>(rows) * static_cast<size_t>(fmt == MXQ_MXFP8 ? K : K / 2);
     return MXQ_OK;
 }
@@ -59,7 +62,7 @@ int validate_quant(const void* x, int64_t M, int64_t K, int fmt, int rule, const
         return MXQ_ERR_UNSUPPORTED;
     if (!x || !q || !sf || (fmt == MXQ_NVFP4 && !g)) return MXQ_ERR_NULL;
     const int bs = block_size(fmt);
-    if (M < 1 || K < bs || K % bs != 0) return MXQ_ERR_SHAPE;
+    if (!dim_ok(M) || !dim_ok(K) || K < bs || K % bs != 0) return MXQ_ERR_SHAPE;
     if (M * K / 8 >= (int64_t(1) << 31)) return MXQ_ERR_SHAPE;  // block indices are 32-bit
     if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || (g && (reinterpret_cast<uintptr_t>(g) & 3u)))
         return MXQ_ERR_ALIGN;
@@ -119,7 +122,7 @@ int mxq_sf_bytes(int64_t rows, int64_t K, mxq_fmt fmt, mxq_sf_layout layout, siz
     if (!valid_fmt(fmt) || (layout != MXQ_SF_ROWMAJOR && layout != MXQ_SF_SWIZZLED)) return MXQ_ERR_UNSUPPORTED;
     if (!bytes) return MXQ_ERR_NULL;
     const int bs = block_size(fmt);
-    if (rows < 1 || K < bs || K % bs != 0) return MXQ_ERR_SHAPE;
+    if (!dim_ok(rows) || !dim_ok(K) || K < bs || K % bs != 0) return MXQ_ERR_SHAPE;
     const int64_t kb = K / bs;
     *bytes = static_cast<size_t>(layout == MXQ_SF_SWIZZLED ? swizzled_sf_bytes(rows, kb) : rows * kb);
     return MXQ_OK;
@@ -220,7 +223,7 @@ int mxq_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxq_fmt fmt) {
 }
 
 size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt) {
-    if (!valid_fmt(fmt) || M < 1 || K < 1 || K % block_size(fmt) != 0) return 0;
+    if (!valid_fmt(fmt) || !dim_ok(M) || !dim_ok(K) || K % block_size(fmt) != 0) return 0;
     size_t qb = 0;
     q_bytes(M, K, fmt, &qb);
     return round256(qb) + static_cast<size_t>(swizzled_sf_bytes(M, K / block_size(fmt)));

@@ -48,6 +48,13 @@ def test_size_helpers(L):
     assert L.mxq_linear_workspace_size(0, 5120, mxq.MXFP4) == 0
     assert L.mxq_linear_kernel_count(32, 5120, 96, mxq.MXFP4) == -2  # K % 64, rejected before any device check
     assert L.mxq_linear_kernel_count(0, 5120, 5120, mxq.MXFP4) == -2
+    # every dimension is bounded (1 <= v < 2^31) before any product of two is formed
+    big = 1 << 40
+    assert L.mxq_sf_bytes(big, big, mxq.MXFP4, mxq.SF_SWIZZLED, ctypes.byref(n)) == -2
+    assert L.mxq_sf_bytes(8, 1 << 31, mxq.MXFP4, mxq.SF_ROWMAJOR, ctypes.byref(n)) == -2
+    assert L.mxq_q_bytes(big, 64, mxq.MXFP4, ctypes.byref(n)) == -2
+    assert L.mxq_linear_workspace_size(big, big, mxq.MXFP4) == 0
+    assert L.mxq_linear_workspace_size((1 << 31) - 1, 64, mxq.MXFP4) > 0
 
 
 def test_host_validation_before_launch(L):
@@ -56,6 +63,8 @@ def test_host_validation_before_launch(L):
     assert L.mxq_quantize(None, 4, 64, 0, 0, None, P, P, 0, s) == -1
     assert L.mxq_quantize(P, 4, 48, 0, 0, None, P, P, 0, s) == -2  # K % 32
     assert L.mxq_quantize(P, 0, 64, 0, 0, None, P, P, 0, s) == -2
+    assert L.mxq_quantize(P, 1 << 40, 1 << 40, 0, 0, None, P, P, 0, s) == -2  # no int64 overflow in M * K
+    assert L.mxq_quantize(P, 1 << 28, 1 << 10, 0, 0, None, P, P, 0, s) == -2  # M * K / 8 >= 2^31
     assert L.mxq_quantize(P + 8, 4, 64, 0, 0, None, P, P, 0, s) == -3
     assert L.mxq_quantize(P, 4, 64, 7, 0, None, P, P, 0, s) == -4
     assert L.mxq_quantize(P, 4, 64, 1, 0, None, P, P, 0, s) == -1  # NVFP4 needs g
