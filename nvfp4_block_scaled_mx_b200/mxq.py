@@ -163,9 +163,33 @@ def sf_bytes(rows, K, fmt, layout=SF_SWIZZLED):
     return n.value
 
 
+def _q_bytes(rows, K, f):
+    return rows * (K if f == MXFP8 else K // 2)
+
+
+def _need(t, name, nbytes, dtype=None):
+    """Host-side guard before a tensor's pointer crosses the C ABI, which sees no sizes: the kernels
+    read or write `nbytes` through it, so a smaller buffer, or one of another element type where
+    the element type matters, is refused here instead of being overrun on the device."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s (got %s)" % (name, dtype, t.dtype))
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError("%s holds %d bytes, the call needs %d" % (name, have, nbytes))
+
+
+def _need_x(x, name="x"):
+    if x.dim() != 2:
+        raise ValueError("%s must be a 2-D [M, K] tensor (got %d dims)" % (name, x.dim()))
+    _need(x, name, 2 * x.numel(), torch.bfloat16)
+
+
 def quantize(x, fmt, rule=EVEN, global_scale=None, layout=SF_SWIZZLED, q_out=None, sf_out=None, stream=None):
     """x [M, K] bf16 (CUDA) -> (q uint8 [M, K/2] or [M, K], sf uint8 flat (swizzled) or [M, K/bs])."""
     f, r = _fmt(fmt), _rule(rule)
+    _need_x(x)
     M, K = x.shape
     if q_out is None:
         q_out = torch.empty(q_shape(M, K, f), dtype=torch.uint8, device=x.device)
@@ -174,6 +198,9 @@ def quantize(x, fmt, rule=EVEN, global_scale=None, layout=SF_SWIZZLED, q_out=Non
             sf_out = torch.empty(sf_bytes(M, K, f, layout), dtype=torch.uint8, device=x.device)
         else:
             sf_out = torch.empty((M, K // block_size(f)), dtype=torch.uint8, device=x.device)
+    _need(q_out, "q_out", _q_bytes(M, K, f))
+    _need(sf_out, "sf_out", sf_bytes(M, K, f, layout))
+    _need(global_scale, "global_scale", 4, torch.float32)
     _check(mxq_quantize(_ptr(x), M, K, f, r, _ptr(global_scale), _ptr(q_out), _ptr(sf_out), layout,
                         _stream(stream)), "mxq_quantize")
     return q_out, sf_out
@@ -181,6 +208,7 @@ def quantize(x, fmt, rule=EVEN, global_scale=None, layout=SF_SWIZZLED, q_out=Non
 
 def quantize_running(x, amax_in, amax_out, layout=SF_SWIZZLED, q_out=None, sf_out=None, stream=None):
     """NVFP4 quantize of x with g = amax_in/2688; amax_out <- max(amax_in, max|x|)."""
+    _need_x(x)
     M, K = x.shape
     if q_out is None:
         q_out = torch.empty(q_shape(M, K, NVFP4), dtype=torch.uint8, device=x.device)
@@ -189,6 +217,10 @@ def quantize_running(x, amax_in, amax_out, layout=SF_SWIZZLED, q_out=None, sf_ou
             sf_out = torch.empty(sf_bytes(M, K, NVFP4, layout), dtype=torch.uint8, device=x.device)
         else:
             sf_out = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+    _need(q_out, "q_out", _q_bytes(M, K, NVFP4))
+    _need(sf_out, "sf_out", sf_bytes(M, K, NVFP4, layout))
+    _need(amax_in, "amax_in", 4, torch.float32)
+    _need(amax_out, "amax_out", 4, torch.float32)
     _check(lib().mxq_quantize_running(_ptr(x), M, K, _ptr(amax_in), _ptr(amax_out), _ptr(q_out), _ptr(sf_out), layout,
                                       _stream(stream)), "mxq_quantize_running")
     return q_out, sf_out
@@ -196,9 +228,12 @@ def quantize_running(x, amax_in, amax_out, layout=SF_SWIZZLED, q_out=None, sf_ou
 
 def fake_quantize(x, fmt, rule=EVEN, global_scale=None, out=None, stream=None):
     """x [M, K] bf16 (CUDA) -> bf16 quantize-dequantize of x (out may be x for in-place)."""
+    _need_x(x)
     M, K = x.shape
     if out is None:
         out = torch.empty_like(x)
+    _need(out, "out", 2 * M * K, torch.bfloat16)
+    _need(global_scale, "global_scale", 4, torch.float32)
     _check(mxq_fake_quantize(_ptr(x), M, K, _fmt(fmt), _rule(rule), _ptr(global_scale), _ptr(out), _stream(stream)),
            "mxq_fake_quantize")
     return out
@@ -206,15 +241,18 @@ def fake_quantize(x, fmt, rule=EVEN, global_scale=None, out=None, stream=None):
 
 def swizzle_scales(sf_rowmajor, out=None, stream=None):
     rows, kb = sf_rowmajor.shape
+    n = ((rows + 127) // 128) * 128 * ((kb + 3) // 4) * 4
     if out is None:
-        n = ((rows + 127) // 128) * 128 * ((kb + 3) // 4) * 4
         out = torch.empty(n, dtype=torch.uint8, device=sf_rowmajor.device)
+    _need(sf_rowmajor, "sf_rowmajor", rows * kb, torch.uint8)
+    _need(out, "out", n)
     _check(mxq_swizzle_scales(_ptr(sf_rowmajor), rows, kb, _ptr(out), _stream(stream)), "mxq_swizzle_scales")
     return out
 
 
 def global_scale(x, stream=None):
     """NVFP4 decode-direction global scale g = amax / 2688 and amax, as device fp32[1] tensors."""
+    _need(x, "x", 2 * x.numel(), torch.bfloat16)
     g = torch.empty(1, dtype=torch.float32, device=x.device)
     amax = torch.empty(1, dtype=torch.float32, device=x.device)
     _check(mxq_global_scale(_ptr(x), x.numel(), _ptr(g), _ptr(amax), _stream(stream)), "mxq_global_scale")
@@ -226,6 +264,13 @@ def gemm(A_q, A_sf, B_q, B_sf, M, N, K, fmt, out_dtype=torch.bfloat16, g_A=None,
     ot = OUT_FP32 if out_dtype == torch.float32 else OUT_BF16
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A_q.device)
+    _need(A_q, "A_q", _q_bytes(M, K, f))
+    _need(B_q, "B_q", _q_bytes(N, K, f))
+    _need(A_sf, "A_sf", sf_bytes(M, K, f))
+    _need(B_sf, "B_sf", sf_bytes(N, K, f))
+    _need(g_A, "g_A", 4, torch.float32)
+    _need(g_B, "g_B", 4, torch.float32)
+    _need(out, "out", M * N * (4 if ot == OUT_FP32 else 2), torch.float32 if ot == OUT_FP32 else torch.bfloat16)
     _check(mxq_gemm(_ptr(A_q), _ptr(A_sf), _ptr(B_q), _ptr(B_sf), _ptr(g_A), _ptr(g_B), M, N, K, f, ot, _ptr(out),
                     _stream(stream)), "mxq_gemm")
     return out
@@ -234,10 +279,15 @@ def gemm(A_q, A_sf, B_q, B_sf, M, N, K, fmt, out_dtype=torch.bfloat16, g_A=None,
 def gemm_w4a16(A, W_q, W_sf, N, fmt, g_W=None, out_dtype=torch.bfloat16, out=None, stream=None):
     """Weight-only GEMM: out = A dq(W)^T with A [M, K] bf16 and W pre-quantized (swizzled scales)."""
     f = _fmt(fmt)
+    _need_x(A, "A")
     M, K = A.shape
     ot = OUT_FP32 if out_dtype == torch.float32 else OUT_BF16
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    _need(W_q, "W_q", _q_bytes(N, K, f))
+    _need(W_sf, "W_sf", sf_bytes(N, K, f))
+    _need(g_W, "g_W", 4, torch.float32)
+    _need(out, "out", M * N * (4 if ot == OUT_FP32 else 2), torch.float32 if ot == OUT_FP32 else torch.bfloat16)
     _check(mxq_gemm_w4a16(_ptr(A), _ptr(W_q), _ptr(W_sf), _ptr(g_W), M, N, K, f, ot, _ptr(out), _stream(stream)),
            "mxq_gemm_w4a16")
     return out
@@ -247,6 +297,7 @@ def linear(x, W_q, W_sf, N, fmt, act_rule=CEIL, out_dtype=torch.bfloat16, g_W=No
            out=None, stream=None):
     """Quantize x per token, then out = A_q W_q^T (W pre-quantized with swizzled scales)."""
     f = _fmt(fmt)
+    _need_x(x)
     M, K = x.shape
     ws = mxq_linear_workspace_size(M, K, f)
     if workspace is None:
@@ -254,6 +305,12 @@ def linear(x, W_q, W_sf, N, fmt, act_rule=CEIL, out_dtype=torch.bfloat16, g_W=No
     ot = OUT_FP32 if out_dtype == torch.float32 else OUT_BF16
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _need(W_q, "W_q", _q_bytes(N, K, f))
+    _need(W_sf, "W_sf", sf_bytes(N, K, f))
+    _need(g_W, "g_W", 4, torch.float32)
+    _need(g_A, "g_A", 4, torch.float32)
+    _need(out, "out", M * N * (4 if ot == OUT_FP32 else 2), torch.float32 if ot == OUT_FP32 else torch.bfloat16)
     _check(mxq_linear(_ptr(x), _ptr(W_q), _ptr(W_sf), _ptr(g_W), _ptr(g_A), M, N, K, f, _rule(act_rule), ot,
-                      _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)), "mxq_linear")
+                      _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+           "mxq_linear")
     return out
