@@ -18,6 +18,7 @@ SF_ROWMAJOR, SF_SWIZZLED = 0, 1
 FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, "mxfp8": MXFP8}
 RULE = {"even": EVEN, "ceil": CEIL}
 
+ERR_SHAPE = -2
 ERR_TIMEOUT = -7
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxq.so")
@@ -51,6 +52,15 @@ class MxqError(RuntimeError):
     def __init__(self, code, where):
         self.code = code
         super().__init__("%s failed: %s (%d)" % (where, lib().mxq_strerror(code).decode(), code))
+
+
+class MxqBufferError(MxqError, ValueError):
+    """A tensor handed to the binding does not fit the call (element type, rank or size); raised
+    before anything reaches the library, with the shape error code."""
+
+    def __init__(self, msg):
+        self.code = ERR_SHAPE
+        Exception.__init__(self, msg)
 
 
 def lib():
@@ -174,15 +184,15 @@ def _need(t, name, nbytes, dtype=None):
     if t is None:
         return
     if dtype is not None and t.dtype != dtype:
-        raise ValueError("%s must be %s (got %s)" % (name, dtype, t.dtype))
+        raise MxqBufferError("%s must be %s (got %s)" % (name, dtype, t.dtype))
     have = t.numel() * t.element_size()
     if have < nbytes:
-        raise ValueError("%s holds %d bytes, the call needs %d" % (name, have, nbytes))
+        raise MxqBufferError("%s holds %d bytes, the call needs %d" % (name, have, nbytes))
 
 
 def _need_x(x, name="x"):
     if x.dim() != 2:
-        raise ValueError("%s must be a 2-D [M, K] tensor (got %d dims)" % (name, x.dim()))
+        raise MxqBufferError("%s must be a 2-D [M, K] tensor (got %d dims)" % (name, x.dim()))
     _need(x, name, 2 * x.numel(), torch.bfloat16)
 
 
@@ -284,6 +294,10 @@ def gemm_w4a16(A, W_q, W_sf, N, fmt, g_W=None, out_dtype=torch.bfloat16, out=Non
     ot = OUT_FP32 if out_dtype == torch.float32 else OUT_BF16
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    if f == MXFP8:  # 4-bit weights only: the library rejects the format before any launch
+        _check(mxq_gemm_w4a16(_ptr(A), _ptr(W_q), _ptr(W_sf), _ptr(g_W), M, N, K, f, ot, _ptr(out), _stream(stream)),
+               "mxq_gemm_w4a16")
+        return out
     _need(W_q, "W_q", _q_bytes(N, K, f))
     _need(W_sf, "W_sf", sf_bytes(N, K, f))
     _need(g_W, "g_W", 4, torch.float32)

@@ -128,3 +128,17 @@ def test_swizzle_scales_sizes(rec):
     with pytest.raises(ValueError, match="sf_rowmajor"):
         mxq.swizzle_scales(torch.zeros(300, 160, dtype=torch.int32))
     assert rec.calls == ["mxq_swizzle_scales"]
+
+
+def test_guard_errors_are_library_errors_too(rec):
+    # callers that catch the library's errors also catch the guards', which carry the shape code
+    with pytest.raises(mxq.MxqError) as e:
+        mxq.quantize(_bf16(4, 64), "mxfp4", q_out=_u8(1))
+    assert e.value.code == mxq.ERR_SHAPE and isinstance(e.value, ValueError)
+    # a W4A16 call with FP8 weights reaches the library, which names the format
+    Wq, Wsf = _u8(8 * 32), _u8(mxq.sf_bytes(8, 64, "mxfp4"))
+    mxq.gemm_w4a16(_bf16(4, 64), Wq, Wsf, 8, "mxfp8")
+    assert rec.calls == ["mxq_gemm_w4a16"]
+    # K = 96 against buffers sized for K = 64: refused on the host
+    with pytest.raises(mxq.MxqError):
+        mxq.gemm_w4a16(_bf16(4, 96), Wq, Wsf, 8, "mxfp4")
