@@ -67,3 +67,51 @@ def test_running_max_oracle(orc):
     g = np.float32(1.0) / np.float32(2688.0)
     q3, sf3 = orc.quantize(x, orc.NVFP4, 0, g=float(g))
     assert np.array_equal(q2, q3) and np.array_equal(sf2, sf3)
+
+
+def _binades(bs, seed):
+    """Two blocks per binade of the block amax, from below the smallest bf16 subnormal to the top of
+    the bf16 range (amax mantissa in [1, 1.4) and in [1.6, 2), so CEIL also moves up a binade)."""
+    g = np.random.default_rng(seed)
+    ks = np.repeat(np.arange(-136, 128), 2)
+    mant = np.where(np.arange(len(ks)) % 2 == 0, 1.0, 1.6) + g.uniform(0.0, 0.39, len(ks))
+    blocks = g.uniform(-1.0, 1.0, (len(ks), bs)) * np.ldexp(1.0, ks)[:, None]
+    blocks[:, 0] = np.ldexp(mant, ks) * g.choice([-1.0, 1.0], len(ks))
+    return torch.from_numpy(blocks.reshape(-1, 128).astype(np.float32)).to(torch.bfloat16)
+
+
+def _bits16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("fmt,rule", [("mxfp4", "even"), ("mxfp4", "ceil"), ("mxfp8", "even"), ("mxfp8", "ceil")])
+def test_mx_fake_quantize_every_scale_code_is_the_bf16_cast(orc, fmt, rule):
+    # every E8M0 code the formats reach (0 through 254): an MX value elem * 2^e has at most 4
+    # significant bits, so its bf16 encoding is torch's bf16 cast of the exact fp64 value (inf where
+    # it exceeds the bf16 range, as a single fp32 product rounds it)
+    f = orc.MXFP4 if fmt == "mxfp4" else orc.MXFP8
+    r = orc.EVEN if rule == "even" else orc.CEIL
+    x = _binades(32, 21)
+    q, sf = orc.quantize(x, f, r)
+    assert sf.min() == 0 and sf.max() >= 246
+    d = orc.dequantize(q, sf, 128, f)
+    expect = _bits16(torch.from_numpy(d).to(torch.bfloat16))
+    assert np.array_equal(orc.fake_quantize(x, f, r), expect)
+
+
+@pytest.mark.parametrize("g", [2.0 ** -140, 1.0e-30, 3.7e-6, 1.0 / 2688, 1.0, 5.0e20, 2.0 ** 100])
+def test_nvfp4_fake_quantize_is_fp32_product_then_bf16(orc, g):
+    # the NVFP4 decode fl32(elem * fl32(dec(s) * g)), then bf16 RNE, rebuilt from library decoders
+    # (ml_dtypes E2M1 and E4M3) and numpy fp32 arithmetic, over blocks in every binade and global
+    # scales that make d subnormal, overflow 1/d, or are plain
+    import ml_dtypes
+    x = _binades(16, 22)
+    g32 = np.float32(g)
+    q, sf = orc.quantize(x, orc.NVFP4, orc.EVEN, g=float(g32))
+    codes = np.stack([q & 0xF, q >> 4], -1).reshape(q.shape[0], -1)
+    elem = codes.astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    dec = sf.view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+    d = (dec * g32).astype(np.float32)
+    prod = (elem * np.repeat(d, 16, axis=1)).astype(np.float32)
+    expect = _bits16(torch.from_numpy(prod).to(torch.bfloat16))
+    assert np.array_equal(orc.fake_quantize(x, orc.NVFP4, orc.EVEN, g=float(g32)), expect)
