@@ -187,7 +187,7 @@ def _nvfp4_reference(x, g):
     s = np.where(amax == 0, np.zeros_like(s), s)
     sdec = s.astype(np.float32)
     d = sdec * g
-    with np.errstate(divide="ignore", invalid="ignore"):
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):  # saturating products are intended
         rcp = np.float32(1.0) / d
         v = b * rcp[..., None]
     codes = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
@@ -324,3 +324,41 @@ def test_gemm_exact_integers(orc):
     part = (ia[0, 32:64] @ ib[:, 32:64].T).astype(np.float64) / 4
     assert np.array_equal(out2[0] - out[0], 7 * part)
     assert np.array_equal(out2[1:], out[1:])
+
+
+def _binades(bs, seed):
+    """Two blocks per binade of the block amax, from below the smallest bf16 subnormal to the top of
+    the bf16 range (amax mantissa in [1, 1.4) and in [1.6, 2), so CEIL also moves up a binade)."""
+    g = np.random.default_rng(seed)
+    ks = np.repeat(np.arange(-136, 128), 2)
+    mant = np.where(np.arange(len(ks)) % 2 == 0, 1.0, 1.6) + g.uniform(0.0, 0.39, len(ks))
+    blocks = g.uniform(-1.0, 1.0, (len(ks), bs)) * np.ldexp(1.0, ks)[:, None]
+    blocks[:, 0] = np.ldexp(mant, ks) * g.choice([-1.0, 1.0], len(ks))
+    return torch.from_numpy(blocks.reshape(-1, 128).astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "mxfp8"])
+@pytest.mark.parametrize("rule", ["even", "ceil"])
+def test_mx_quantize_every_scale_code_matches_library_construction(orc, fmt, rule):
+    # every E8M0 code the rules reach, 0 through 254, including the clamp at -127 for subnormal
+    # blocks and the top binade of bf16
+    f = orc.MXFP4 if fmt == "mxfp4" else orc.MXFP8
+    r = orc.EVEN if rule == "even" else orc.CEIL
+    x = _binades(32, 31)
+    q, sf = orc.quantize(x, f, r)
+    codes_ref, sf_ref = _mx_reference(x, fmt, rule)
+    assert np.array_equal(sf, sf_ref)
+    assert sf.min() == 0 and sf.max() >= 246
+    codes = q if fmt == "mxfp8" else _unpack_fp4(q)
+    assert np.array_equal(codes, codes_ref)
+
+
+@pytest.mark.parametrize("g", [1.0e-30, 3.7e-6, 1.0 / 2688, 1.0, 5.0e20, 2.0 ** 100])
+def test_nvfp4_every_binade_matches_fp32_library_construction(orc, g):
+    # blocks in every binade against fixed global scales that send scales to 0, saturate them at
+    # 448, or leave them in range (subnormal g, where fl(1/d) can overflow, is pinned separately)
+    x = _binades(16, 32)
+    q, sf = orc.quantize(x, orc.NVFP4, 0, g=g)
+    codes_ref, sf_ref = _nvfp4_reference(x, g)
+    assert np.array_equal(sf, sf_ref)
+    assert np.array_equal(_unpack_fp4(q), codes_ref)
