@@ -106,8 +106,19 @@ int mxq_quantize_running(const void* x_bf16, int64_t M, int64_t K, const float* 
 int mxq_fake_quantize(const void* x_bf16, int64_t M, int64_t K, mxq_fmt fmt, mxq_rule rule, const float* global_scale,
                       void* y_bf16, mxq_stream_t stream);
 
-/* Re-lay row-major scales [rows, kblocks] (device) into the swizzled tensor-core layout
- * (device, mxq_sf_bytes(SWIZZLED) bytes, padding zeroed).  Pure byte permutation. */
+/*
+ * Re-lay row-major scales [rows, kblocks] (device) into the swizzled tensor-core layout
+ * (device, mxq_sf_bytes(SWIZZLED) bytes, padding zeroed).  Pure byte permutation.
+ * The pages do not describe this layout: they only store the scales as U8 tensors
+ * ("intel-ai/Qwen3.8-27B-MXFP4-AutoRound", section 1 "Model summary", Weight dtype row) that the
+ * serving FP4 kernel consumes.  The layout is
+ * the one the tcgen05 block-scaled MMA reads its scale factors in (128-row x 4-column tiles, see the
+ * conventions above); this library's own reading, confirmed end to end by the GEMM parity tests.
+ *   sf_rowmajor  (device) rows * kblocks bytes, read only.
+ *   sf_swizzled  (device) mxq_sf_bytes(rows, K, fmt, MXQ_SF_SWIZZLED) bytes, written whole.
+ * Errors: MXQ_ERR_NULL for a NULL pointer, MXQ_ERR_SHAPE unless 1 <= rows < 2^31 and
+ * 1 <= kblocks < 2^24; nothing is launched then.
+ */
 int mxq_swizzle_scales(const uint8_t* sf_rowmajor, int64_t rows, int64_t kblocks, uint8_t* sf_swizzled,
                        mxq_stream_t stream);
 
@@ -117,6 +128,16 @@ int mxq_swizzle_scales(const uint8_t* sf_rowmajor, int64_t rows, int64_t kblocks
  * running-max form of input_global_scale ("Qwen3.5-27B-NVFP4-GPTQ", Serving-KL table, RTN row).
  */
 int mxq_global_scale(const void* x_bf16, int64_t n, float* g_out, float* amax_out, mxq_stream_t stream);
+
+/*
+ * Tensor amax of x (n bf16 values, device, 16-byte aligned): *amax_out = max |x| (device fp32[1],
+ * exact: a bf16 value is an fp32 value).  This is the tensor-max helper a caller uses to derive a
+ * dynamic NVFP4 global scale or to feed a running-max observer ("Qwen3.5-27B-NVFP4-GPTQ",
+ * Serving-KL table: running-max versus static input scales); mxq_global_scale is the same
+ * reduction followed by g = fl(amax / (6 * 448)).  Errors: MXQ_ERR_NULL, MXQ_ERR_SHAPE (n < 1),
+ * MXQ_ERR_ALIGN; nothing is launched then.  Stream-ordered; allocates nothing.
+ */
+int mxq_amax(const void* x_bf16, int64_t n, float* amax_out, mxq_stream_t stream);
 
 /*
  * Block-scaled GEMM on the tcgen05 tensor cores: out[M, N] = alpha * dq(A) dq(B)^T, fp32
@@ -165,18 +186,32 @@ size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt);
 int mxq_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxq_fmt fmt);
 
 /*
- * Quantized linear layer: quantize x [M, K] bf16 per token with act_rule (MX) or global scale g_A
- * (NVFP4, device fp32[1]) into `workspace`, then out = A_q * W_q^T through mxq_gemm.
- * W_q / W_sf are the pre-quantized weights (SWIZZLED scales), g_W their NVFP4 global scale.
- * The activation quantizer and the GEMM run back to back on `stream` with programmatic
- * dependent launch; A is quantized once, not once per output tile.
+ * Quantized linear layer, the W4A4 serving path: the activations are quantized dynamically per
+ * token at run time and multiplied with the pre-quantized weights by an FP4 GEMM
+ * ("Qwen3.5-9B-MXFP4-QAD-W4A4-LR1e-5-s3000", Serving, W4A4 bullet; the CEIL activation rule from its
+ * "Training mode" paragraph).  out = dq(Q(x)) dq(W)^T * alpha with Q the quantizer of mxq_quantize.
+ *   x_bf16     (device) [M, K] bf16 activations, row-major.
+ *   W_q, W_sf  (device) the pre-quantized weights [N, K] (mxq_quantize output) with SWIZZLED scales.
+ *   g_W, g_A   (device) fp32[1] NVFP4 global scales of W and of x (decode direction); ignored (may
+ *              be NULL) for MX formats.
+ *   act_rule   MX scale rule of the activations (ignored for NVFP4).
+ *   workspace  (device) at least mxq_linear_workspace_size(M, K, fmt) bytes, caller-owned, 16-byte
+ *              aligned: the quantized activations and their swizzled scales (up to 32 tokens the
+ *              call may not touch it).
+ *   out        (device) [M, N] bf16 (RNE) or fp32, row-major.
+ * Requirements as mxq_gemm, plus M * K / 8 < 2^31.  The quantizer and the GEMM run back to back on
+ * `stream` with programmatic dependent launch (one launch up to 32 tokens, see
+ * mxq_linear_kernel_count); A is quantized once, not once per output tile.  Errors are checked in
+ * this order before anything is launched: MXQ_ERR_UNSUPPORTED (fmt, act_rule, out_type),
+ * MXQ_ERR_NULL, MXQ_ERR_SHAPE, MXQ_ERR_ALIGN, MXQ_ERR_WORKSPACE (ws_bytes too small),
+ * MXQ_ERR_DEVICE; MXQ_ERR_CUDA reports a failed launch.
  */
 int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
                int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule, mxq_out out_type,
                void* workspace, size_t ws_bytes, void* out, mxq_stream_t stream);
 
 /*
- * mxq_linear without a caller-supplied workspace.  The paper has no counterpart: this call exists
+ * mxq_linear without a caller-supplied workspace.  The pages have no counterpart: this call exists
  * for callers that are not allowed to allocate device memory -- e.g. plugins inside a host
  * framework that owns all device memory and passes only input and output buffers, or processes
  * under a fixed device-memory cap that must not grow (or synchronise the device through an
@@ -186,8 +221,10 @@ int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const f
  * bytes per GPU, held by every GPU that loads the library until the process exits.  Problems
  * whose mxq_linear_workspace_size(M, K, fmt) exceeds that size are rejected with
  * MXQ_ERR_WORKSPACE before anything is launched (8 MiB covers, e.g., up to 2048 tokens at K = 5120
- * for FP4).  Other arguments, requirements and results are exactly those of mxq_linear; the caller
- * still provides x, the quantized weights and `out`.  The call allocates nothing.
+ * for FP4).  Other arguments, requirements, error codes (in mxq_linear's order, the scratch limit
+ * taking the place of the workspace size) and results are exactly those of mxq_linear: the same
+ * kernels on the same bytes, so the output is bit-identical.  The caller still provides x, the
+ * quantized weights and `out`.  The call allocates nothing.
  *
  * The first call on a device looks up the array's device address (once per device, with that
  * device current); make that first call before any stream capture.  All calls share the one array

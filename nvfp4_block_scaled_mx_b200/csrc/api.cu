@@ -27,6 +27,8 @@ bool valid_fmt(int fmt) { return fmt == MXQ_MXFP4 || fmt == MXQ_NVFP4 || fmt == 
 bool valid_rule(int rule) { return rule == MXQ_RULE_EVEN || rule == MXQ_RULE_CEIL; }
 bool valid_out(int out) { return out == MXQ_OUT_BF16 || out == MXQ_OUT_FP32; }
 
+}  // namespace
+
 // Checks the current device is an sm_100 part (the library carries sm_100a code only).
 int check_device() {
     static std::atomic<int> verdict[kMaxDevices];
@@ -43,6 +45,8 @@ int check_device() {
     }
     return v == 1 ? MXQ_OK : MXQ_ERR_DEVICE;
 }
+
+namespace {
 
 // A dimension the library accepts: 1 <= v < 2^31 (products of two fit in 62 bits).
 bool dim_ok(int64_t v) { return v >= 1 && v < (int64_t(1) << 31); }
@@ -101,6 +105,37 @@ int sm_count() {
         counts[dev].store(c);
     }
     return c;
+}
+
+int validate_linear(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
+                    int64_t M, int64_t N, int64_t K, int fmt, int act_rule, int out_type, const void* out,
+                    bool caller_workspace, const void* workspace) {
+    if (!valid_fmt(fmt) || !valid_out(out_type) || (fmt != MXQ_NVFP4 && !valid_rule(act_rule)))
+        return MXQ_ERR_UNSUPPORTED;
+    if (!x || !W_q || !W_sf || !out || (caller_workspace && !workspace) || (fmt == MXQ_NVFP4 && (!g_W || !g_A)))
+        return MXQ_ERR_NULL;
+    int rc = validate_gemm_shape(M, N, K, fmt);
+    if (rc != MXQ_OK) return rc;
+    if (M * K / 8 >= (int64_t(1) << 31)) return MXQ_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(W_q) || !aligned16(W_sf) || !aligned16(out) ||
+        (caller_workspace && !aligned16(workspace)))
+        return MXQ_ERR_ALIGN;
+    return MXQ_OK;
+}
+
+int run_linear(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A, int64_t M,
+               int64_t N, int64_t K, int fmt, int act_rule, int out_type, void* workspace, void* out,
+               cudaStream_t st) {
+    size_t qb = 0;
+    q_bytes(M, K, fmt, &qb);
+    uint8_t* a_q = static_cast<uint8_t*>(workspace);
+    uint8_t* a_sf = a_q + round256(qb);
+    // few tokens: one launch, the GEMM quantizing its own activations (the workspace stays unused)
+    int rc = launch_linear_fused(x, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, out, st);
+    if (rc != kNotFused) return rc;
+    if (launch_quantize(x, M, K, fmt, act_rule, g_A, a_q, a_sf, MXQ_SF_SWIZZLED, st) != cudaSuccess)
+        return MXQ_ERR_CUDA;
+    return launch_gemm(a_q, a_sf, W_q, W_sf, g_A, g_W, M, N, K, fmt, out_type, out, st, true);
 }
 
 }  // namespace mxq
@@ -189,6 +224,17 @@ int mxq_global_scale(const void* x_bf16, int64_t n, float* g_out, float* amax_ou
                : MXQ_ERR_CUDA;
 }
 
+int mxq_amax(const void* x_bf16, int64_t n, float* amax_out, mxq_stream_t stream) {
+    if (!x_bf16 || !amax_out) return MXQ_ERR_NULL;
+    if (n < 1) return MXQ_ERR_SHAPE;
+    if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(amax_out) & 3u)) return MXQ_ERR_ALIGN;
+    int rc = check_device();
+    if (rc != MXQ_OK) return rc;
+    return launch_global_scale(x_bf16, n, nullptr, amax_out, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MXQ_OK
+               : MXQ_ERR_CUDA;
+}
+
 int mxq_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uint8_t* B_sf, const float* g_A,
              const float* g_B, int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_out out_type, void* out,
              mxq_stream_t stream) {
@@ -232,27 +278,12 @@ size_t mxq_linear_workspace_size(int64_t M, int64_t K, mxq_fmt fmt) {
 int mxq_linear(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
                int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule, mxq_out out_type, void* workspace,
                size_t ws_bytes, void* out, mxq_stream_t stream) {
-    if (!valid_fmt(fmt) || !valid_out(out_type) || (fmt != MXQ_NVFP4 && !valid_rule(act_rule)))
-        return MXQ_ERR_UNSUPPORTED;
-    if (!x_bf16 || !W_q || !W_sf || !out || !workspace || (fmt == MXQ_NVFP4 && (!g_W || !g_A))) return MXQ_ERR_NULL;
-    int rc = validate_gemm_shape(M, N, K, fmt);
+    int rc = validate_linear(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, out, true, workspace);
     if (rc != MXQ_OK) return rc;
-    if (M * K / 8 >= (int64_t(1) << 31)) return MXQ_ERR_SHAPE;
-    if (!aligned16(x_bf16) || !aligned16(W_q) || !aligned16(W_sf) || !aligned16(out) || !aligned16(workspace))
-        return MXQ_ERR_ALIGN;
     if (ws_bytes < mxq_linear_workspace_size(M, K, fmt)) return MXQ_ERR_WORKSPACE;
     if ((rc = check_device()) != MXQ_OK) return rc;
-    size_t qb = 0;
-    q_bytes(M, K, fmt, &qb);
-    uint8_t* a_q = static_cast<uint8_t*>(workspace);
-    uint8_t* a_sf = a_q + round256(qb);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // few tokens: one launch, the GEMM quantizing its own activations (the workspace stays unused)
-    rc = launch_linear_fused(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, out, st);
-    if (rc != kNotFused) return rc;
-    if (launch_quantize(x_bf16, M, K, fmt, act_rule, g_A, a_q, a_sf, MXQ_SF_SWIZZLED, st) != cudaSuccess)
-        return MXQ_ERR_CUDA;
-    return launch_gemm(a_q, a_sf, W_q, W_sf, g_A, g_W, M, N, K, fmt, out_type, out, st, true);
+    return run_linear(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, workspace, out,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int mxq_device_status(int* status_out, int reset, mxq_stream_t stream) {

@@ -34,7 +34,10 @@ int scratch_address(void** out) {
     void* p = g_scratch_addr[dev].load();
     if (p == nullptr) {
         void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, mxq_noalloc_scratch) != cudaSuccess || addr == nullptr) return MXQ_ERR_CUDA;
+        if (cudaGetSymbolAddress(&addr, mxq_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+            (void)cudaGetLastError();  // clear the runtime's last error: the return code reports it
+            return MXQ_ERR_CUDA;
+        }
         g_scratch_addr[dev].store(addr);
         p = addr;
     }
@@ -47,15 +50,17 @@ int scratch_address(void** out) {
 extern "C" int mxq_linear_noalloc(const void* x_bf16, const void* W_q, const uint8_t* W_sf, const float* g_W,
                                   const float* g_A, int64_t M, int64_t N, int64_t K, mxq_fmt fmt, mxq_rule act_rule,
                                   mxq_out out_type, void* out, mxq_stream_t stream) {
-    const size_t need = mxq_linear_workspace_size(M, K, fmt);
-    if (need == 0) return MXQ_ERR_SHAPE;
-    if (need > static_cast<size_t>(MXQ_NOALLOC_SCRATCH_BYTES)) return MXQ_ERR_WORKSPACE;
-    void* ws = nullptr;
-    const int rc = scratch_address(&ws);
+    // the argument checks of mxq_linear, in its order, then the scratch limit in place of the
+    // caller's workspace size, then the device: the same codes mxq_linear returns for the same inputs
+    int rc = mxq::validate_linear(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, out, false, nullptr);
     if (rc != MXQ_OK) return rc;
+    if (mxq_linear_workspace_size(M, K, fmt) > static_cast<size_t>(MXQ_NOALLOC_SCRATCH_BYTES)) return MXQ_ERR_WORKSPACE;
+    if ((rc = mxq::check_device()) != MXQ_OK) return rc;
+    void* ws = nullptr;
+    if ((rc = scratch_address(&ws)) != MXQ_OK) return rc;
     // Everything the GEMM reads from the scratch is rewritten by this call's quantizer (codes of
     // all M rows, scales including their zero padding), so the previous call's contents never leak
     // into the result.
-    return mxq_linear(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, ws,
-                      static_cast<size_t>(MXQ_NOALLOC_SCRATCH_BYTES), out, stream);
+    return mxq::run_linear(x_bf16, W_q, W_sf, g_W, g_A, M, N, K, fmt, act_rule, out_type, ws, out,
+                           reinterpret_cast<cudaStream_t>(stream));
 }

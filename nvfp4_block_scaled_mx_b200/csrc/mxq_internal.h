@@ -12,6 +12,22 @@ namespace mxq {
 // Device status word of the current device (kernels record bounded-wait timeouts there).
 int* status_ptr();
 
+// MXQ_OK if the current device is an sm_100 part, MXQ_ERR_DEVICE otherwise (MXQ_ERR_CUDA when the
+// query fails); cached per device.
+int check_device();
+
+// Host-side argument checks of the linear layer, in mxq_linear's order (unsupported enum, NULL
+// pointer, shape, alignment); the workspace pointer is checked only when the caller supplies one.
+int validate_linear(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
+                    int64_t M, int64_t N, int64_t K, int fmt, int act_rule, int out_type, const void* out,
+                    bool caller_workspace, const void* workspace);
+
+// The linear layer's launches on validated arguments: the one-launch few-token path, else the
+// quantizer into `workspace` (mxq_linear_workspace_size bytes) followed by the GEMM.
+int run_linear(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A, int64_t M,
+               int64_t N, int64_t K, int fmt, int act_rule, int out_type, void* workspace, void* out,
+               cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
@@ -39,6 +55,8 @@ cudaError_t launch_fake_quantize(const void* x, int64_t M, int64_t K, int fmt, i
 
 cudaError_t launch_swizzle(const uint8_t* src, int64_t rows, int64_t kblocks, uint8_t* dst, cudaStream_t stream);
 
+// Tensor amax of n bf16 values into *amax_out, then g = fl(amax / 2688) into *g_out (skipped when
+// g_out is NULL).
 cudaError_t launch_global_scale(const void* x, int64_t n, float* g_out, float* amax_out, cudaStream_t stream);
 
 // GEMM launch.  `pdl_secondary` launches with programmatic stream serialization so that the

@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
                     int64_t n_units, uint32_t kblocks, uint64_t kb_magic,
                     uint32_t col_tiles, const float* __restrict__ gptr, uint8_t* __restrict__ q,
                     uint8_t* __restrict__ sf, unsigned int* __restrict__ amax_out, int* status,
-                    const void* __restrict__ x_tail, bool tail) {
+                    const void* __restrict__ x_tail, bool tail, uint32_t rows) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(ring + kQuantStages * kQuantStageBytes);
@@ -208,6 +208,28 @@ __global__ void __launch_bounds__(kQuantBoxThreads, kQuantCtasPerSm)
             if (b >= n_boxes) break;
             mbar_arrive_expect_tx(&full[st], kQuantStageBytes);
             tma_load_2d(&tmap_x, &full[st], ring + st * kQuantStageBytes, 0, static_cast<int>(b * kQuantRows), pol);
+        }
+    }
+    if constexpr (SWZ && !FAKE) {
+        // The swizzled layout's padding is zero: rows M .. (M rounded up to 128) of the last row
+        // tile, and scale columns kblocks .. (kblocks rounded up to 4) of every row.  The main loop
+        // never writes these bytes, so the grid zeroes them here, while the first boxes load.
+        const uint32_t cols = col_tiles * 4u;
+        const uint32_t pad_cols = cols - kblocks;
+        const uint64_t n_row_pad = static_cast<uint64_t>(((rows + 127u) & ~127u) - rows) * cols;
+        const uint64_t n_pad = n_row_pad + static_cast<uint64_t>(rows) * pad_cols;
+        for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_pad;
+             i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+            uint32_t r, c;
+            if (i < n_row_pad) {
+                r = rows + static_cast<uint32_t>(i / cols);
+                c = static_cast<uint32_t>(i % cols);
+            } else {
+                const uint64_t j = i - n_row_pad;  // only reached when pad_cols > 0
+                r = static_cast<uint32_t>(j / pad_cols);
+                c = kblocks + static_cast<uint32_t>(j % pad_cols);
+            }
+            sf[swz_offset(r, c, col_tiles)] = 0;
         }
     }
     const float g = (FMT == MXQ_NVFP4) ? (OBS ? __fdiv_rn(*gptr, 2688.0f) : *gptr) : 1.0f;
@@ -366,7 +388,8 @@ cudaError_t launch_q_tma(const void* x, int64_t M, int64_t K, const float* g, vo
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, tmap, tmap_y, n_units, kblocks, kb_magic, col_tiles, g, static_cast<uint8_t*>(q),
                               static_cast<uint8_t*>(sf), amax_out, status_ptr(),
-                              static_cast<const void*>(static_cast<const uint8_t*>(x) + n_units * 64), tail);
+                              static_cast<const void*>(static_cast<const uint8_t*>(x) + n_units * 64), tail,
+                              static_cast<uint32_t>(M));
 }
 
 template <int FMT, int RULE, bool SWZ>
@@ -451,14 +474,7 @@ __global__ void selftest_timeout_kernel(int* status, uint64_t limit_ns) {
 
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int fmt, int rule, const float* g, void* q, void* sf,
                             int layout, cudaStream_t stream) {
-    if (layout == MXQ_SF_SWIZZLED) {
-        const int64_t kb = K / block_size(fmt);
-        if (M % 128 != 0 || kb % 4 != 0) {
-            cudaError_t e = cudaMemsetAsync(sf, 0, static_cast<size_t>(swizzled_sf_bytes(M, kb)), stream);
-            if (e != cudaSuccess) return e;
-        }
-        return launch_q_layout<true>(x, M, K, fmt, rule, g, q, sf, stream);
-    }
+    if (layout == MXQ_SF_SWIZZLED) return launch_q_layout<true>(x, M, K, fmt, rule, g, q, sf, stream);
     return launch_q_layout<false>(x, M, K, fmt, rule, g, q, sf, stream);
 }
 
@@ -477,14 +493,7 @@ cudaError_t launch_quantize_running(const void* x, int64_t M, int64_t K, const f
     // amax_out starts from the running state, then takes this batch's maximum
     cudaError_t e = cudaMemcpyAsync(amax_out, amax_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
     if (e != cudaSuccess) return e;
-    if (layout == MXQ_SF_SWIZZLED) {
-        const int64_t kb = K / 16;
-        if (M % 128 != 0 || kb % 4 != 0) {
-            e = cudaMemsetAsync(sf, 0, static_cast<size_t>(swizzled_sf_bytes(M, kb)), stream);
-            if (e != cudaSuccess) return e;
-        }
-        return launch_q_running<true>(x, M, K, amax_in, amax_out, q, sf, stream);
-    }
+    if (layout == MXQ_SF_SWIZZLED) return launch_q_running<true>(x, M, K, amax_in, amax_out, q, sf, stream);
     return launch_q_running<false>(x, M, K, amax_in, amax_out, q, sf, stream);
 }
 
@@ -511,7 +520,7 @@ cudaError_t launch_global_scale(const void* x, int64_t n, float* g_out, float* a
         static_cast<const uint4*>(x), n_chunks, static_cast<const uint16_t*>(x) + n_chunks * 8, n_tail,
         reinterpret_cast<unsigned int*>(amax_out));
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || g_out == nullptr) return e;  // mxq_amax stops at the tensor amax
     global_scale_finalize<<<1, 1, 0, stream>>>(amax_out, g_out);
     return cudaGetLastError();
 }

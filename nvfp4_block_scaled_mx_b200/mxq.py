@@ -34,6 +34,7 @@ SIGNATURES = {
     "mxq_fake_quantize": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P]),
     "mxq_swizzle_scales": (_I, [_P, _I64, _I64, _P, _P]),
     "mxq_global_scale": (_I, [_P, _I64, _P, _P, _P]),
+    "mxq_amax": (_I, [_P, _I64, _P, _P]),
     "mxq_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_gemm_w4a16": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _P]),
     "mxq_linear_workspace_size": (_SZ, [_I64, _I64, _I]),
@@ -121,6 +122,10 @@ def mxq_swizzle_scales(sf_rowmajor, rows, kblocks, sf_swizzled, stream):
 
 def mxq_global_scale(x, n, g_out, amax_out, stream):
     return lib().mxq_global_scale(x, n, g_out, amax_out, stream)
+
+
+def mxq_amax(x, n, amax_out, stream):
+    return lib().mxq_amax(x, n, amax_out, stream)
 
 
 def mxq_gemm(A_q, A_sf, B_q, B_sf, g_A, g_B, M, N, K, fmt, out_type, out, stream):
@@ -267,6 +272,14 @@ def global_scale(x, stream=None):
     amax = torch.empty(1, dtype=torch.float32, device=x.device)
     _check(mxq_global_scale(_ptr(x), x.numel(), _ptr(g), _ptr(amax), _stream(stream)), "mxq_global_scale")
     return g, amax
+
+
+def amax(x, stream=None):
+    """max |x| over the whole tensor, as a device fp32[1] tensor."""
+    _need(x, "x", 2 * x.numel(), torch.bfloat16)
+    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(mxq_amax(_ptr(x), x.numel(), _ptr(out), _stream(stream)), "mxq_amax")
+    return out
 
 
 def gemm(A_q, A_sf, B_q, B_sf, M, N, K, fmt, out_dtype=torch.bfloat16, g_A=None, g_B=None, out=None, stream=None):

@@ -77,4 +77,28 @@ def test_host_validation_before_launch(L):
     assert L.mxq_swizzle_scales(None, 4, 4, P, s) == -1
     assert L.mxq_global_scale(P, 0, P, P, s) == -2
     assert L.mxq_selftest_timeout(0, s) == -2
+    assert L.mxq_amax(None, 4, P, s) == -1
+    assert L.mxq_amax(P, 0, P, s) == -2
+    assert L.mxq_amax(P + 8, 4, P, s) == -3
+    # the allocation-free linear call reports mxq_linear's codes in mxq_linear's order
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 4, 4, 128, 7, 1, 0, P, s) == -4
+    assert L.mxq_linear_noalloc(None, P, P, None, None, 4, 4, 128, 0, 1, 0, P, s) == -1
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 4, 4, 96, 0, 1, 0, P, s) == -2
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 8192, 4, 5120, 0, 1, 0, P, s) == -5
+    assert L.mxq_linear(P, P, P, None, None, 4, 4, 128, 7, 1, 0, P, 1 << 20, P, s) == -4
     assert L.mxq_strerror(-5) == b"workspace too small"
+
+
+# the calls of the method's hot path: each declaration's comment names the page (a quoted title)
+# that defines the operation, or says that the pages do not describe it
+CITED = ["mxq_quantize", "mxq_quantize_running", "mxq_fake_quantize", "mxq_swizzle_scales", "mxq_global_scale",
+         "mxq_amax", "mxq_gemm", "mxq_gemm_w4a16", "mxq_linear"]
+
+
+def test_header_cites_the_defining_passage():
+    txt = open(os.path.join(ROOT, "include", "mxq.h")).read()
+    for name in CITED:
+        m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*(?:#define[^\n]*\n\s*)?int %s\(" % name, txt, flags=re.S)
+        assert m, "no comment block directly above %s" % name
+        comment = m.group(1)
+        assert re.search(r'"(Qwen3\.5|intel-ai)[^"]*"', comment.replace("\n *", " ")), "%s cites no page" % name

@@ -1,5 +1,5 @@
-"""Out-of-bounds writes, checked with canaries (a stand-in for compute-sanitizer, which this pool
-does not offer): every output buffer of a call sits inside a larger allocation, 4 KB from its start
+"""Out-of-bounds writes, checked with canaries (a stand-in for a memory-checking tool, which these
+tests do not run): every output buffer of a call sits inside a larger allocation, 4 KB from its start
 (keeping 16-byte alignment), whose bytes outside the buffer hold a sentinel pattern; after the call,
 not one of them may have changed.  Shapes are those of the parity tests: ragged M, N and K tails, a
 single element, several tiles, and both the one-launch and the two-launch linear paths."""
@@ -77,3 +77,30 @@ def test_gemm_and_linear_write_inside_their_output(fmt, M, N, K, out_dtype):
         mxq.gemm_w4a16(A, Wq, Wsf, N, fmt, g_W=g_w, out_dtype=out_dtype, out=o3.t)
         torch.cuda.synchronize()
         assert o3.intact(), "W4A16 output written outside its buffer"
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("M,N,K", [(17, 300, 320), (129, 520, 1024), (300, 257, 576)])
+def test_noalloc_writes_inside_its_output(fmt, M, N, K):
+    """The allocation-free linear entry point writes its quantized activations into a static array
+    of the library, next to its other device globals; an overrun there would corrupt them unseen.
+    Its output must stay inside its canaried buffer, the device status word must stay clean, and a
+    regular mxq_linear afterwards must still give the same bytes."""
+    A = synth.random_bf16((M, K), 7 * M + K, device="cuda")
+    W = synth.random_bf16((N, K), 11 * N + K, std=0.02, device="cuda")
+    g_a = g_w = None
+    if fmt == "nvfp4":
+        g_a, g_w = mxq.global_scale(A)[0], mxq.global_scale(W)[0]
+    Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w)
+    mxq.mxq_device_status(reset=True)
+    o = Canary(M * N * 2, torch.bfloat16, (M, N))
+    p = lambda t: None if t is None else t.data_ptr()
+    rc = mxq.lib().mxq_linear_noalloc(p(A), p(Wq), p(Wsf), p(g_w), p(g_a), M, N, K, mxq.FMT[fmt], mxq.CEIL,
+                                      mxq.OUT_BF16, p(o.t), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert o.intact(), "no-alloc linear output written outside its buffer"
+    assert mxq.mxq_device_status(reset=True) == 0
+    expect = mxq.linear(A, Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=torch.bfloat16, g_W=g_w, g_A=g_a)
+    torch.cuda.synchronize()
+    assert torch.equal(o.t.view(torch.int16), expect.view(torch.int16))

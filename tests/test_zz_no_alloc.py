@@ -4,9 +4,10 @@ Callers that may not allocate device memory (plugins that only receive their inp
 buffers, processes under a fixed device-memory cap) use mxq_linear_noalloc, which takes the
 activation workspace from a static array inside the library instead of from the caller.  These
 tests call it through the C ABI and check its output against the regular mxq_linear on the same
-inputs, within the GEMM tolerance used by every other parity test, for two calls in a row (the
-second with fewer tokens and different data, so stale scratch contents would show).  This file
-is collected last on purpose: a failure here leaves every other test already run.
+inputs for two calls in a row (the second with fewer tokens and different data, so stale scratch
+contents would show).  Both calls run the same kernels on the same bytes, so the outputs must be
+bit-identical; the oracle's GEMM tolerance is checked as well.  This file is collected last on
+purpose: a failure here leaves every other test already run.
 """
 import ctypes
 
@@ -48,17 +49,19 @@ def test_noalloc_matches_linear_two_calls(fmt, out_dtype):
         out = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
         assert _noalloc(A, Wq, Wsf, N, fmt, "ceil", out, g_w, g_a) == 0
         torch.cuda.synchronize()
-        # sum_k |a_k b_k| from the oracle sets the tolerance scale
+        # the oracle from the bf16 inputs, with the tolerance of every other parity test
         gA = float(g_a.item()) if g_a is not None else 1.0
         gW = float(g_w.item()) if g_w is not None else 1.0
         Aq, Asf = oracle_quantize(A.cpu(), fmt, "ceil", gA)
-        _, abs_sum = oracle.gemm(Aq, Asf, Wq_ref, Wsf_ref, M, N, K, FMTS[fmt], gA=gA, gB=gW)
-        got, ref = out.double().cpu().numpy(), expect.double().cpu().numpy()
+        bits = torch.int32 if out_dtype == torch.float32 else torch.int16
+        assert torch.equal(out.view(bits), expect.view(bits)), "noalloc differs from mxq_linear at M=%d" % M
+        ref, abs_sum = oracle.gemm(Aq, Asf, Wq_ref, Wsf_ref, M, N, K, FMTS[fmt], gA=gA, gB=gW)
+        got = out.double().cpu().numpy()
         assert np.isfinite(got).all()
         if out_dtype == torch.float32:
-            check_fp32(got, ref, abs_sum, "noalloc vs linear M=%d" % M)
+            check_fp32(got, ref, abs_sum, "noalloc vs oracle M=%d" % M)
         else:
-            check_bf16(got, ref, abs_sum, "noalloc vs linear M=%d" % M)
+            check_bf16(got, ref, abs_sum, "noalloc vs oracle M=%d" % M)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
@@ -69,3 +72,15 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     Wsf = torch.empty(mxq.sf_bytes(N, K, "mxfp4"), dtype=torch.uint8, device="cuda")
     out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     assert _noalloc(x, Wq, Wsf, N, "mxfp4", "ceil", out) == -5  # MXQ_ERR_WORKSPACE, nothing launched
+
+
+def test_noalloc_error_codes_match_linear():
+    """Bad arguments give mxq_linear's codes, in its order, before anything is launched or looked
+    up: an unknown format is MXQ_ERR_UNSUPPORTED (not a shape error)."""
+    P = 0x10000  # never dereferenced: every case fails validation first
+    L = mxq.lib()
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 4, 4, 128, 7, 1, 0, P, None) == -4
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 4, 4, 128, 0, 9, 0, P, None) == -4
+    assert L.mxq_linear_noalloc(None, P, P, None, None, 4, 4, 128, 0, 1, 0, P, None) == -1
+    assert L.mxq_linear_noalloc(P, P, P, None, None, 4, 4, 96, 0, 1, 0, P, None) == -2
+    assert L.mxq_linear_noalloc(P + 8, P, P, None, None, 4, 4, 128, 0, 1, 0, P, None) == -3
