@@ -327,6 +327,8 @@ def run_mxq(args, world, rank, local):
         e2e = run_e2e(lambda a, o, st: mxq.linear(a, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype,
                                                   g_W=g_w, g_A=g_a, workspace=ws, out=o, stream=st),
                       A, out, flops, args, world, dev)
+    # full-size bf16 inputs for the oracle quantizer timing of the CPU baseline (rank 0, N = 1)
+    host_inputs = (A.cpu(), W.cpu()) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else (None, None)
     others = None
     if not args.no_others and world == 1:
         del A, W, W_q, W_sf, ws, out
@@ -343,7 +345,7 @@ def run_mxq(args, world, rank, local):
            "gpu_launches": mxq.linear_kernel_count(M, N, K, fmt) * args.steps, "roofline": roofline, "quantize": quant, "quantize_weight": quant_w,
            "fake_quantize": fake_quant,
            "clocks": clk.summary(), "e2e": e2e, "other_workloads": others}
-    return res
+    return res, host_inputs
 
 
 def other_workloads(stream, bf16_tflops):
@@ -488,33 +490,65 @@ def oracle_sample(workload, rows, cols, seed=0):
     return cfg, A, W
 
 
-def oracle_step(orc, cfg, A, Wq, Wsf, gW):
+def oracle_step(orc, cfg, A, Wq, Wsf, gW, threads=1):
     fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
     rules = {"even": orc.EVEN, "ceil": orc.CEIL}
     f = fmts[cfg["fmt"]]
     gA = 1.0
     if cfg["fmt"] == "nvfp4":
         gA, _ = orc.global_scale(A)
-    Aq, Asf = orc.quantize(A, f, rules[cfg["a_rule"]], g=float(gA))
-    orc.gemm(Aq, Asf, Wq, Wsf, A.shape[0], Wq.shape[0], cfg["K"], f, gA=float(gA), gB=float(gW))
+    Aq, Asf = orc.quantize(A, f, rules[cfg["a_rule"]], g=float(gA), threads=threads)
+    orc.gemm(Aq, Asf, Wq, Wsf, A.shape[0], Wq.shape[0], cfg["K"], f, gA=float(gA), gB=float(gW), threads=threads)
 
 
-def cpu_baseline(workload, rows=256, cols=4096):
+def cpu_baseline(workload, A_full=None, W_full=None, rows=128, cols=4096):
+    """The oracle as it stands, timed on this host's cores: the linear step (quantize a sample of
+    activation rows + fp64 GEMM against a sample of quantized weight rows) on one thread and on every
+    usable CPU (one POSIX thread per range of output columns), and the oracle quantizer's GB/s over
+    the full activation and weight tensors of the workload (all CPUs; activations also on one
+    thread).  About 10-30 s of CPU work on a many-core host."""
     import oracle as orc
+    orc.build()
     cfg, A, W = oracle_sample(workload, rows, cols)
     fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
     rules = {"even": orc.EVEN, "ceil": orc.CEIL}
+    f = fmts[cfg["fmt"]]
+    usable, online = orc.cpus_usable(), orc.cpus_online()
     gW = 1.0
     if cfg["fmt"] == "nvfp4":
         gW, _ = orc.global_scale(W)
-    Wq, Wsf = orc.quantize(W, fmts[cfg["fmt"]], rules[cfg["w_rule"]], g=float(gW))
-    t0 = time.perf_counter()
-    oracle_step(orc, cfg, A, Wq, Wsf, gW)
-    dt = time.perf_counter() - t0
+    Wq, Wsf = orc.quantize(W, f, rules[cfg["w_rule"]], g=float(gW), threads=usable)
     flops = 2.0 * rows * cols * cfg["K"]
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": "%d activation rows x %d weight rows x K=%d of %s: CEIL/EVEN quantize of the rows + fp64 "
-                      "GEMM, single-threaded scalar C, %.1f s" % (rows, cols, cfg["K"], workload, dt)}
+    rates = {}
+    for threads in (1, usable):
+        t0 = time.perf_counter()
+        oracle_step(orc, cfg, A, Wq, Wsf, gW, threads=threads)
+        dt = time.perf_counter() - t0
+        rates[threads] = (flops / dt / 1e12, dt)
+    res = {"value": rates[usable][0], "unit": "TFLOP/s", "cores": usable, "host_cpus_online": online,
+           "kind": "oracle",
+           "sample": "%d activation rows x %d weight rows x K=%d of %s: %s quantize of the rows + fp64 GEMM, "
+                     "scalar C on %d threads (%.2f s); host has %d online CPUs, %d usable" % (
+                         rows, cols, cfg["K"], workload, cfg["a_rule"].upper(), usable, rates[usable][1], online,
+                         usable),
+           "single_thread": {"value": rates[1][0], "unit": "TFLOP/s", "cores": 1, "seconds": round(rates[1][1], 2)}}
+    qres = {}
+    bpe = QUANT_BYTES_PER_ELEM[cfg["fmt"]]
+    for which, x, rule, thread_counts in (("activations", A_full, cfg["a_rule"], (1, usable)),
+                                          ("weights", W_full, cfg["w_rule"], (usable,))):
+        if x is None:
+            continue
+        g = float(orc.global_scale(x)[0]) if cfg["fmt"] == "nvfp4" else 1.0
+        r = {"shape": list(x.shape), "rule": rule}
+        for threads in thread_counts:
+            t0 = time.perf_counter()
+            orc.quantize(x, f, rules[rule], g=g, threads=threads)
+            dt = time.perf_counter() - t0
+            r["gbs_%s" % ("1_thread" if threads == 1 else "%d_threads" % threads)] = round(bpe * x.numel() / dt / 1e9, 3)
+        qres[which] = r
+    if qres:
+        res["quantize_full_tensors"] = qres
+    return res
 
 
 def run_reference(args, world, rank):
@@ -522,6 +556,7 @@ def run_reference(args, world, rank):
         return None
     import oracle as orc
     orc.build()
+    threads = orc.cpus_usable()
     rows, cols = 8, 512
     cfg, A, W = oracle_sample(args.workload, rows, cols)
     fmts = {"mxfp4": orc.MXFP4, "nvfp4": orc.NVFP4, "mxfp8": orc.MXFP8}
@@ -529,23 +564,24 @@ def run_reference(args, world, rank):
     gW = 1.0
     if cfg["fmt"] == "nvfp4":
         gW, _ = orc.global_scale(W)
-    Wq, Wsf = orc.quantize(W, fmts[cfg["fmt"]], rules[cfg["w_rule"]], g=float(gW))
+    Wq, Wsf = orc.quantize(W, fmts[cfg["fmt"]], rules[cfg["w_rule"]], g=float(gW), threads=threads)
     for _ in range(max(1, args.warmup)):
-        oracle_step(orc, cfg, A, Wq, Wsf, gW)
+        oracle_step(orc, cfg, A, Wq, Wsf, gW, threads=threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(orc, cfg, A, Wq, Wsf, gW)
+        oracle_step(orc, cfg, A, Wq, Wsf, gW, threads=threads)
     dt = time.perf_counter() - t0
     flops = 2.0 * rows * cols * cfg["K"]
     value = flops * args.steps / dt / 1e12
     sample = ("per step %d activation rows x %d weight rows x K=%d of %s (quantize rows + fp64 GEMM), "
-              "scalar C oracle, 1 thread" % (rows, cols, cfg["K"], args.workload))
+              "scalar C oracle on %d threads (host: %d online CPUs)" % (rows, cols, cfg["K"], args.workload, threads,
+                                                                        orc.cpus_online()))
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": {"workload": args.workload, "M": cfg["M"], "N": cfg["N"],
                                                      "K": cfg["K"], "fmt": cfg["fmt"]},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -670,9 +706,9 @@ def main():
         if args.impl == "reference":
             res = run_reference(args, world, rank)
         else:
-            res = run_mxq(args, world, rank, local)
-            if rank == 0 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline(args.workload)
+            res, host_inputs = run_mxq(args, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(args.workload, *host_inputs)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -35,13 +35,22 @@
  * (ml_dtypes, torch), exact rational arithmetic or brute force, except the NVFP4 operation order
  * and the MXFP8 scale rule, which are readings (the pages do not fix them).
  *
- * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -o liboracle.so mxq_oracle.c -lm
+ * Threads: orc_quantize_mt and orc_gemm_mt split the rows (quantizer) or the output columns (GEMM)
+ * into contiguous ranges, one per POSIX thread, each running exactly the single-threaded code on its
+ * range; every output value is computed by the same operations in the same order as with one
+ * thread, so the results do not depend on the thread count.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -pthread -ffp-contract=off -o liboracle.so mxq_oracle.c -lm
  * (no -ffast-math: fp32 steps must be plain IEEE operations).
  */
+#define _GNU_SOURCE
 #include <math.h>
+#include <pthread.h>
+#include <sched.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <unistd.h>
 
 #define ORC_MXFP4 0
 #define ORC_NVFP4 1
@@ -227,6 +236,76 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t K, int fmt, int rule, 
     return 0;
 }
 
+/* ---------------------------------------------------------------- threads */
+
+/* Logical CPUs this process may run on (its affinity mask), and the host's online CPU count. */
+int orc_cpus_usable(void) {
+    cpu_set_t set;
+    CPU_ZERO(&set);
+    if (sched_getaffinity(0, sizeof set, &set) == 0) {
+        int n = CPU_COUNT(&set);
+        if (n > 0) return n;
+    }
+    return 1;
+}
+
+int orc_cpus_online(void) {
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+typedef struct {
+    const uint16_t* x;
+    int64_t rows, K;
+    int fmt, rule;
+    float g;
+    uint8_t *q, *sf;
+    int rc;
+} quant_job;
+
+static void* quant_worker(void* arg) {
+    quant_job* j = (quant_job*)arg;
+    j->rc = orc_quantize(j->x, j->rows, j->K, j->fmt, j->rule, j->g, j->q, j->sf);
+    return NULL;
+}
+
+/* orc_quantize over `nthreads` POSIX threads, each quantizing a contiguous range of rows (rows are
+ * independent).  Same bytes as orc_quantize.  Returns 0, or -1 as orc_quantize, or -2 when a
+ * thread cannot be created. */
+int orc_quantize_mt(const uint16_t* x, int64_t rows, int64_t K, int fmt, int rule, float g, uint8_t* q,
+                    uint8_t* sf, int nthreads) {
+    int bs = fmt_block(fmt);
+    if (K % bs != 0) return -1;
+    if (nthreads > rows) nthreads = (int)rows;
+    if (nthreads <= 1) return orc_quantize(x, rows, K, fmt, rule, g, q, sf);
+    int64_t qrow = fmt == ORC_MXFP8 ? K : K / 2, kb = K / bs;
+    quant_job* jobs = (quant_job*)calloc((size_t)nthreads, sizeof(quant_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) {
+        free(jobs);
+        free(th);
+        return -2;
+    }
+    int started = 0, rc = 0;
+    for (int t = 0; t < nthreads; t++) {
+        int64_t r0 = rows * t / nthreads, r1 = rows * (t + 1) / nthreads;
+        quant_job j = {x + r0 * K, r1 - r0, K, fmt, rule, g, q + r0 * qrow, sf + r0 * kb, 0};
+        jobs[t] = j;
+        if (pthread_create(&th[t], NULL, quant_worker, &jobs[t]) != 0) {
+            rc = -2;
+            break;
+        }
+        started++;
+    }
+    for (int t = 0; t < started; t++) {
+        pthread_join(th[t], NULL);
+        if (jobs[t].rc != 0 && rc == 0) rc = jobs[t].rc;
+    }
+    free(jobs);
+    free(th);
+    return rc;
+}
+
 /* Decoded value of element (r, k) of a quantized matrix, without the NVFP4 global scale. */
 static double dq_elem(const uint8_t* q, const uint8_t* sf, int64_t r, int64_t k, int64_t K, int fmt) {
     int bs = fmt_block(fmt);
@@ -292,42 +371,102 @@ float orc_global_scale(const uint16_t* x, int64_t n, float* amax_out) {
 /* Out[i][j] = alpha * sum_k dq(A)[rows[i]][k] * dq(B)[cols[j]][k] in fp64, alpha = gA*gB for
  * NVFP4 and 1 otherwise; abs_out[i][j] = |alpha| * sum_k |dq(A) dq(B)|.  A is [M][K], B is [N][K]
  * (nn.Linear layout), both quantized along K with row-major scales.  rows / cols select which
- * outputs to compute (pass NULL for all).  Returns 0. */
-int orc_gemm(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Bq, const uint8_t* Bsf, double gA,
-             double gB, int64_t M, int64_t N, int64_t K, int fmt, const int64_t* rows, int64_t nrows,
-             const int64_t* cols, int64_t ncols, double* out, double* abs_out) {
+ * outputs to compute (pass NULL for all).  Each sum runs over k in increasing order. */
+typedef struct {
+    const uint8_t *Bq, *Bsf;
+    const double* arow; /* dequantized selected A rows, [nrows][K] */
+    const int64_t* cols;
+    int64_t K, nrows, ncols, j0, j1;
+    int fmt;
+    double alpha;
+    double *out, *abs_out;
+    int rc;
+} gemm_job;
+
+static void* gemm_cols(void* arg) {
+    gemm_job* g = (gemm_job*)arg;
+    int64_t K = g->K;
+    double* brow = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!brow) {
+        g->rc = -1;
+        return NULL;
+    }
+    for (int64_t j = g->j0; j < g->j1; j++) {
+        int64_t n = g->cols ? g->cols[j] : j;
+        for (int64_t k = 0; k < K; k++) brow[k] = dq_elem(g->Bq, g->Bsf, n, k, K, g->fmt);
+        for (int64_t i = 0; i < g->nrows; i++) {
+            double acc = 0.0, aacc = 0.0;
+            const double* a = g->arow + i * K;
+            for (int64_t k = 0; k < K; k++) {
+                double p = a[k] * brow[k];
+                acc += p;
+                aacc += fabs(p);
+            }
+            g->out[i * g->ncols + j] = g->alpha * acc;
+            if (g->abs_out) g->abs_out[i * g->ncols + j] = fabs(g->alpha) * aacc;
+        }
+    }
+    free(brow);
+    g->rc = 0;
+    return NULL;
+}
+
+/* The GEMM over `nthreads` POSIX threads, each taking a contiguous range of the selected output
+ * columns.  Returns 0, or -1 when memory runs out or a thread cannot be created. */
+int orc_gemm_mt(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Bq, const uint8_t* Bsf, double gA,
+                double gB, int64_t M, int64_t N, int64_t K, int fmt, const int64_t* rows, int64_t nrows,
+                const int64_t* cols, int64_t ncols, double* out, double* abs_out, int nthreads) {
     double alpha = fmt == ORC_NVFP4 ? gA * gB : 1.0;
     if (!rows) nrows = M;
     if (!cols) ncols = N;
+    if (nthreads > ncols) nthreads = (int)ncols;
+    if (nthreads < 1) nthreads = 1;
     double* arow = (double*)malloc(sizeof(double) * (size_t)(nrows * K));
-    double* brow = (double*)malloc(sizeof(double) * (size_t)K);
-    if (!arow || !brow) {
+    gemm_job* jobs = (gemm_job*)calloc((size_t)nthreads, sizeof(gemm_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!arow || !jobs || !th) {
         free(arow);
-        free(brow);
+        free(jobs);
+        free(th);
         return -1;
     }
     for (int64_t i = 0; i < nrows; i++) {
         int64_t m = rows ? rows[i] : i;
         for (int64_t k = 0; k < K; k++) arow[i * K + k] = dq_elem(Aq, Asf, m, k, K, fmt);
     }
-    for (int64_t j = 0; j < ncols; j++) {
-        int64_t n = cols ? cols[j] : j;
-        for (int64_t k = 0; k < K; k++) brow[k] = dq_elem(Bq, Bsf, n, k, K, fmt);
-        for (int64_t i = 0; i < nrows; i++) {
-            double acc = 0.0, aacc = 0.0;
-            const double* a = arow + i * K;
-            for (int64_t k = 0; k < K; k++) {
-                double p = a[k] * brow[k];
-                acc += p;
-                aacc += fabs(p);
+    int rc = 0, started = 0;
+    for (int t = 0; t < nthreads; t++) {
+        gemm_job j = {Bq, Bsf, arow, cols, K, nrows, ncols, ncols * t / nthreads, ncols * (t + 1) / nthreads,
+                      fmt, alpha, out, abs_out, 0};
+        jobs[t] = j;
+    }
+    if (nthreads == 1) {
+        gemm_cols(&jobs[0]);
+        rc = jobs[0].rc;
+    } else {
+        for (int t = 0; t < nthreads; t++) {
+            if (pthread_create(&th[t], NULL, gemm_cols, &jobs[t]) != 0) {
+                rc = -1;
+                break;
             }
-            out[i * ncols + j] = alpha * acc;
-            if (abs_out) abs_out[i * ncols + j] = fabs(alpha) * aacc;
+            started++;
+        }
+        for (int t = 0; t < started; t++) {
+            pthread_join(th[t], NULL);
+            if (jobs[t].rc != 0) rc = -1;
         }
     }
     free(arow);
-    free(brow);
-    return 0;
+    free(jobs);
+    free(th);
+    return rc;
+}
+
+/* The GEMM on one thread.  Returns 0, or -1 when memory runs out. */
+int orc_gemm(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Bq, const uint8_t* Bsf, double gA,
+             double gB, int64_t M, int64_t N, int64_t K, int fmt, const int64_t* rows, int64_t nrows,
+             const int64_t* cols, int64_t ncols, double* out, double* abs_out) {
+    return orc_gemm_mt(Aq, Asf, Bq, Bsf, gA, gB, M, N, K, fmt, rows, nrows, cols, ncols, out, abs_out, 1);
 }
 
 /* Weight-only (W4A16) GEMM, the serving mode of "Qwen3.5-27B-NVFP4-RTN-weight-only" (first paragraph:

@@ -22,7 +22,7 @@ def build(force=False):
     """Compile the oracle with plain gcc (IEEE fp32/fp64, no contraction, no fast-math)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".%d.tmp" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
                                "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -50,6 +50,11 @@ def lib():
         L.orc_global_scale.argtypes, L.orc_global_scale.restype = [p, i64, p], f
         L.orc_gemm.argtypes = [p, p, p, p, d, d, i64, i64, i64, i32, p, i64, p, i64, p, p]
         L.orc_gemm.restype = i32
+        L.orc_gemm_mt.argtypes = [p, p, p, p, d, d, i64, i64, i64, i32, p, i64, p, i64, p, p, i32]
+        L.orc_gemm_mt.restype = i32
+        L.orc_quantize_mt.argtypes, L.orc_quantize_mt.restype = [p, i64, i64, i32, i32, f, p, p, i32], i32
+        L.orc_cpus_usable.argtypes, L.orc_cpus_usable.restype = [], i32
+        L.orc_cpus_online.argtypes, L.orc_cpus_online.restype = [], i32
         L.orc_gemm_w4a16.argtypes = [p, p, p, d, i64, i64, i64, i32, p, i64, p, i64, p, p]
         L.orc_gemm_w4a16.restype = i32
         L.orc_f32_to_bf16.argtypes, L.orc_f32_to_bf16.restype = [f], ctypes.c_uint16
@@ -108,17 +113,34 @@ def _bits(x):
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
-def quantize(x, fmt, rule=EVEN, g=1.0):
+def cpus_usable():
+    """Logical CPUs this process may run on (its affinity mask)."""
+    return lib().orc_cpus_usable()
+
+
+def cpus_online():
+    """Online logical CPUs of the host."""
+    return lib().orc_cpus_online()
+
+
+def _threads(threads):
+    return cpus_usable() if threads is None else max(1, int(threads))
+
+
+def quantize(x, fmt, rule=EVEN, g=1.0, threads=1):
     """x: [rows, K] bf16 -> (q, sf).  q: [rows, K/2] uint8 (FP4, low nibble first) or [rows, K]
-    (MXFP8); sf: [rows, K/bs] uint8 row-major scale codes."""
+    (MXFP8); sf: [rows, K/bs] uint8 row-major scale codes.  threads: row ranges quantized in
+    parallel (None = every usable CPU); the bytes do not depend on it."""
     xb = _bits(x)
     rows, K = xb.shape
     bs = block_size(fmt)
     q = np.zeros((rows, K if fmt == MXFP8 else K // 2), dtype=np.uint8)
     sf = np.zeros((rows, K // bs), dtype=np.uint8)
-    rc = lib().orc_quantize(_ptr(xb), rows, K, fmt, rule, float(g), _ptr(q), _ptr(sf))
-    if rc != 0:
+    rc = lib().orc_quantize_mt(_ptr(xb), rows, K, fmt, rule, float(g), _ptr(q), _ptr(sf), _threads(threads))
+    if rc == -1:
         raise ValueError("K=%d is not a multiple of the block size %d" % (K, bs))
+    if rc != 0:
+        raise RuntimeError("oracle quantize could not start its threads")
     return q, sf
 
 
@@ -162,9 +184,10 @@ def global_scale(x):
     return np.float32(g), np.float32(amax.value)
 
 
-def gemm(Aq, Asf, Bq, Bsf, M, N, K, fmt, gA=1.0, gB=1.0, rows=None, cols=None):
+def gemm(Aq, Asf, Bq, Bsf, M, N, K, fmt, gA=1.0, gB=1.0, rows=None, cols=None, threads=1):
     """fp64 reference of Out = alpha * dq(A) @ dq(B)^T on the selected rows/cols.
-    Returns (out, abs_sum), both [len(rows), len(cols)] float64."""
+    Returns (out, abs_sum), both [len(rows), len(cols)] float64.  threads: output column ranges
+    computed in parallel (None = every usable CPU); the values do not depend on it."""
     Aq, Asf, Bq, Bsf = (np.ascontiguousarray(a, dtype=np.uint8) for a in (Aq, Asf, Bq, Bsf))
     r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
@@ -172,9 +195,9 @@ def gemm(Aq, Asf, Bq, Bsf, M, N, K, fmt, gA=1.0, gB=1.0, rows=None, cols=None):
     nc = N if c is None else c.size
     out = np.zeros((nr, nc), dtype=np.float64)
     absout = np.zeros((nr, nc), dtype=np.float64)
-    rc = lib().orc_gemm(_ptr(Aq), _ptr(Asf), _ptr(Bq), _ptr(Bsf), float(gA), float(gB), M, N, K, fmt,
-                        None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
-                        _ptr(out), _ptr(absout))
+    rc = lib().orc_gemm_mt(_ptr(Aq), _ptr(Asf), _ptr(Bq), _ptr(Bsf), float(gA), float(gB), M, N, K, fmt,
+                           None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
+                           _ptr(out), _ptr(absout), _threads(threads))
     if rc != 0:
         raise MemoryError("oracle gemm allocation failed")
     return out, absout

@@ -202,12 +202,37 @@ def test_bounded_wait_selftest():
     assert int(sf[0, 0]) == 125  # amax 1 -> CEIL e = -2
 
 
+# fixed seeds of the sampled rows and columns, one per problem (reproducible across processes)
+SAMPLE_SEED = {"decode": 2001, "prefill_gate_up": 2002, "down_nvfp4": 2003, "attn_mxfp8": 2004, "lm_head": 2005,
+               "in_proj_ba": 2006}
+
+
+def _sample(total, tile, n, gen):
+    """About n seeded indices in [0, total): the same number in every `tile`-wide stretch (at least
+    one), so every output tile the kernels emit is visited, plus the last index (the tail)."""
+    if total <= n:
+        return np.arange(total, dtype=np.int64)
+    tiles = (total + tile - 1) // tile
+    per = max(1, -(-n // tiles))
+    idx = set()
+    for t in range(tiles):
+        lo, hi = t * tile, min(total, (t + 1) * tile)
+        idx.update(torch.randint(lo, hi, (min(per, hi - lo),), generator=gen).tolist())
+    idx.add(total - 1)
+    return np.array(sorted(idx), dtype=np.int64)
+
+
 @pytest.mark.parametrize("name", ["decode", "prefill_gate_up", "down_nvfp4", "attn_mxfp8", "lm_head", "in_proj_ba"])
-def test_linear_full_size_sampled(name):
+def test_linear_full_size(name):
     """Each full-size problem through mxq_linear in the bench's launch configuration (weights
-    quantized on the GPU, activations quantized inside the call); a seeded sample of outputs
-    (random rows x random columns plus the last row and column) is recomputed by the oracle from
-    the bf16 inputs alone."""
+    quantized on the GPU, activations quantized inside the call), checked against the oracle run on
+    the bf16 inputs alone:
+      - every quantized byte of A and W (mxq_quantize, the quantizer mxq_linear runs) equals the
+        oracle's;
+      - outputs: about 128 seeded rows (the same number in every 256-row M tile, plus the last row)
+        times ALL N columns, and ALL M rows times about 128 seeded columns (the same number in every
+        256-column N tile, plus the last column); every output when M or N is small (decode: all of
+        it).  Together they visit every output tile, the last partial waves and the N tail."""
     cfg = synth.CONFIGS[name]
     M, N, K, fmt = cfg["M"], cfg["N"], cfg["K"], cfg["fmt"]
     A, W = synth.make_inputs(name, device="cuda")
@@ -223,15 +248,31 @@ def test_linear_full_size_sampled(name):
     Wq, Wsf = mxq.quantize(W, fmt, cfg["w_rule"], global_scale=g_w, layout=mxq.SF_SWIZZLED)
     out_dtype = torch.float32 if cfg["out"] == "fp32" else torch.bfloat16
     out = mxq.linear(A, Wq, Wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+    Aq_gpu, Asf_gpu = mxq.quantize(A, fmt, cfg["a_rule"], global_scale=g_a, layout=mxq.SF_SWIZZLED)
     torch.cuda.synchronize()
-    gen = torch.Generator().manual_seed(hash(name) % 1000)
-    rows = sorted(set(torch.randint(0, M, (min(M, 48),), generator=gen).tolist()) | {M - 1})
-    cols = sorted(set(torch.randint(0, N, (48,), generator=gen).tolist()) | {N - 1})
-    Aq, Asf = oracle_quantize(A[rows].cpu(), fmt, cfg["a_rule"], gA)
-    Wq_ref, Wsf_ref = oracle_quantize(W[cols].cpu(), fmt, cfg["w_rule"], gW)
-    ref, abs_sum = oracle.gemm(Aq, Asf, Wq_ref, Wsf_ref, len(rows), len(cols), K, FMTS[fmt], gA=gA, gB=gW)
-    gpu = out[rows][:, cols].double().cpu().numpy()
-    if out_dtype == torch.float32:
-        check_fp32(gpu, ref, abs_sum, name)
-    else:
-        check_bf16(gpu, ref, abs_sum, name)
+    assert mxq.mxq_device_status(reset=True) == 0
+    bs = 16 if fmt == "nvfp4" else 32
+
+    # every quantized byte of both operands (oracle threads over row ranges; the bytes do not depend on it)
+    Wq_ref, Wsf_ref = oracle.quantize(W.cpu(), FMTS[fmt], RULES[cfg["w_rule"]], g=gW, threads=None)
+    assert np.array_equal(to_np(Wq), Wq_ref), "%s: weight codes differ" % name
+    assert np.array_equal(to_np(Wsf), oracle.swizzle(Wsf_ref)), "%s: weight scales differ" % name
+    Aq_ref, Asf_ref = oracle.quantize(A.cpu(), FMTS[fmt], RULES[cfg["a_rule"]], g=gA, threads=None)
+    assert np.array_equal(to_np(Aq_gpu), Aq_ref), "%s: activation codes differ" % name
+    assert np.array_equal(to_np(Asf_gpu), oracle.swizzle(Asf_ref)), "%s: activation scales differ" % name
+    del Wq, Wsf, Aq_gpu, Asf_gpu, W, A
+
+    check = check_fp32 if out_dtype == torch.float32 else check_bf16
+    gen = torch.Generator().manual_seed(SAMPLE_SEED[name])
+    rows = _sample(M, 256, 128, gen)
+    cols = _sample(N, 256, 128, gen)
+    # seeded rows x all columns
+    ref, abs_sum = oracle.gemm(Aq_ref, Asf_ref, Wq_ref, Wsf_ref, M, N, K, FMTS[fmt], gA=gA, gB=gW, rows=rows,
+                               threads=None)
+    check(out[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref, abs_sum, "%s rows x all N" % name)
+    if len(rows) < M:
+        # all rows x seeded columns, as the transposed product (the fp64 sums are the same terms)
+        ref_t, abs_t = oracle.gemm(Wq_ref, Wsf_ref, Aq_ref, Asf_ref, N, M, K, FMTS[fmt], gA=gW, gB=gA, rows=cols,
+                                   threads=None)
+        check(out[:, torch.from_numpy(cols).cuda()].double().cpu().numpy(), ref_t.T, abs_t.T,
+              "%s all M x columns" % name)
