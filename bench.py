@@ -291,15 +291,28 @@ def run_mxq(args, world, rank, local):
                 "frac_of_datasheet": round(gemm_tflops / (9000.0 if fmt != "mxfp8" else 4500.0), 4),
                 "traffic": traffic_for("gemm_%s_%s" % (fmt, workload)),
                 "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
-    if M <= 128:
-        # few tokens: the GEMM streams its weights once (HBM-bound); timed with the L2 flushed
-        gemm_cold = time_flushed(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a,
-                                                  g_B=g_w, out=out, stream=stream), 20, stream, flush)
-        gbytes = W_q.numel() + W_sf.numel() + a_q.numel() + a_sf.numel() + out.numel() * out.element_size()
-        roofline = {"bound": "hbm", "kernel": "gemm_splitk_kernel / gemm_kernel (tcgen05 kind::%s, few tokens)" % kind,
-                    "achieved": round(gbytes / gemm_cold / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
-                    "frac": round(gbytes / gemm_cold / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
-                    "traffic": None, "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(gemm_cold * 1e3, 4),
+    one_launch = mxq.linear_kernel_count(M, N, K, fmt) == 1
+    if M <= 128 or one_launch:
+        # few tokens or few columns: the layer streams its weights (few tokens) or its bf16 activations
+        # (few columns) once and is HBM-bound.  Timed with the L2 flushed before each launch, as the
+        # linear call itself when that is one launch (the GEMM quantizing its own activations: bf16
+        # rows in), else as the GEMM on quantized activations
+        if one_launch:
+            lin_cold = time_flushed(lambda: mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype,
+                                                       g_W=g_w, g_A=g_a, workspace=ws, out=out, stream=stream),
+                                    20, stream, flush)
+            gbytes = W_q.numel() + W_sf.numel() + 2 * M * K + out.numel() * out.element_size()
+            kname = ("gemm_splitk_kernel (tcgen05 kind::%s, few tokens, activations quantized in the kernel)" if M <= 32
+                     else "gemm_rowq_kernel (tcgen05 kind::%s, few columns, activations quantized in the kernel)") % kind
+        else:
+            lin_cold = time_flushed(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a,
+                                                     g_B=g_w, out=out, stream=stream), 20, stream, flush)
+            gbytes = W_q.numel() + W_sf.numel() + a_q.numel() + a_sf.numel() + out.numel() * out.element_size()
+            kname = "gemm_splitk_kernel / gemm_kernel (tcgen05 kind::%s, few tokens)" % kind
+        roofline = {"bound": "hbm", "kernel": kname,
+                    "achieved": round(gbytes / lin_cold / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
+                    "frac": round(gbytes / lin_cold / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
+                    "traffic": None, "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(lin_cold * 1e3, 4),
                     "l2": "flushed per launch (the launch latency is inside the time)"}
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),

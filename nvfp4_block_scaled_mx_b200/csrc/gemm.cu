@@ -777,6 +777,663 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ few-token linear kernel
+//
+// The decode-shaped linear layer (up to 32 tokens): streaming the weights is the whole cost, so a
+// CTA owns 128 weight rows and a contiguous share of the K stages (the S CTAs of a cluster split K
+// and reduce through distributed shared memory), and everything else hides under the weight
+// stream.  The weights are the MMA's 128-row A operand and the tokens its N = 32 columns, so the
+// accumulator is 32 TMEM columns whose 128 lanes span all four sub-partitions.  The bf16 tokens are
+// quantized inside the kernel, in a ring of their own that runs ahead of the weight ring: the
+// quantization of the first stages overlaps the latency of the first weight loads instead of
+// following their arrival.
+//   warp 0       TMA producer of the weight ring (codes, 128 rows x 128 bytes; their scale tiles)
+//   warp 1       TMEM owner; copies each stage's weight and token scale tiles into TMEM
+//                (tcgen05.cp) and issues the MMAs
+//   warp 2       TMA producer of the bf16 token ring (boxes of 64 elements x 32 rows, 128B swizzle)
+//   warps 3-10   quantize the token stages into the token-code ring (B operand layout) with the
+//                streaming quantizer's arithmetic; then the epilogue.  Partials of the non-leader
+//                CTAs go to a buffer of their own in the leader as soon as they are ready.
+template <int KIND>
+struct DecCfg {
+    static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
+    static constexpr int BK = 128 * EPB;
+    static constexpr int KSTEPS = BK / MMA_K;
+    static constexpr int KB_PER_MMA = MMA_K / BS;
+    static constexpr int SF_ATOMS = BK / BS / 4;
+    static constexpr int TOK = 32;                   // MMA N: token rows (rows >= M are zero)
+    static constexpr int WSTAGES = 5, XSTAGES = 3, TSTAGES = 6;
+    static constexpr int W_BYTES = 128 * 128;
+    static constexpr int SF_BYTES = SF_ATOMS * 512;
+    static constexpr int X_BOXES = BK / 64;
+    static constexpr int X_BYTES = X_BOXES * TOK * 128;
+    static constexpr int T_BYTES = TOK * 128;
+    static constexpr int QWARPS = 8;
+    static constexpr int THREADS = (3 + QWARPS) * 32;
+    static constexpr int RED_BYTES = (kMaxSplits - 1) * 128 * TOK * 4;
+    static constexpr int OFF_W = 0;
+    static constexpr int OFF_X = OFF_W + WSTAGES * W_BYTES;
+    static constexpr int OFF_T = OFF_X + XSTAGES * X_BYTES;
+    static constexpr int OFF_RED = OFF_T + TSTAGES * T_BYTES;
+    static constexpr int OFF_SFW = OFF_RED + RED_BYTES;
+    static constexpr int OFF_SFT = OFF_SFW + WSTAGES * SF_BYTES;
+    static constexpr int OFF_TAB = OFF_SFT + TSTAGES * SF_BYTES;
+    static constexpr int OFF_BAR = OFF_TAB + 1024;
+    static constexpr int N_BARS = 2 * (WSTAGES + XSTAGES + TSTAGES) + 2;  // + accf, rfull
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
+    static constexpr int SLOT_COLS = 2 * SF_ATOMS * 4;  // per weight stage: weight then token scale tiles
+    static constexpr int SF_TMEM_BASE = 32;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static_assert(KSTEPS == 4, "4 MMAs per stage");
+    static_assert(SF_TMEM_BASE + WSTAGES * SLOT_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
+    static_assert(OFF_W % 1024 == 0 && OFF_X % 1024 == 0 && OFF_T % 1024 == 0, "swizzled buffers 1024-aligned");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int KIND, bool OUT_F32, int QRULE>
+__global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_w,
+                       const GemmArgs p) {
+    using C = DecCfg<KIND>;
+    constexpr int WS = C::WSTAGES, XS = C::XSTAGES, TS = C::TSTAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* wempty = wfull + WS;
+    uint64_t* xfull = wempty + WS;
+    uint64_t* xempty = xfull + XS;
+    uint64_t* tready = xempty + XS;
+    uint64_t* tempty = tready + TS;
+    uint64_t* accf = tempty + TS;
+    uint64_t* rfull = accf + 1;  // leader: every partial has landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+    float* tab_d = reinterpret_cast<float*>(smem + C::OFF_TAB);
+    float* tab_r = tab_d + 128;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t split = cluster_ctarank();
+    const uint32_t splits = p.k_split;
+    const int nt = static_cast<int>(blockIdx.x / splits);
+    const int per = (p.k_stages + static_cast<int>(splits) - 1) / static_cast<int>(splits);
+    const int k0 = static_cast<int>(split) * per;
+    const int k1 = min(p.k_stages, k0 + per);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_x);
+        prefetch_tmap(&tma_w);
+        for (int s = 0; s < WS; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], 1);
+        }
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], C::QWARPS);
+        }
+        for (int s = 0; s < TS; ++s) {
+            mbar_init(&tready[s], C::QWARPS);
+            mbar_init(&tempty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(rfull, 1);
+        // the other splits - 1 CTAs' partials (128 weight rows x 32 tokens, fp32), counted in bytes
+        if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * 128u * C::TOK * 4u);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_arrive_relaxed();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
+
+    if (warp == 0) {
+        // weight producer: the whole warp runs the loop; one elected lane issues
+        const uint64_t pol = policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&wempty[stage], phase ^ 1u, p.status, 51)) break;
+            if (elect_one()) {
+                const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
+                mbar_arrive_expect_tx(&wfull[stage], C::W_BYTES + atoms * 512);
+                tma_load_2d(&tma_w, &wfull[stage], smem + C::OFF_W + stage * C::W_BYTES, ks * 128, nt * 128, pol);
+                bulk_load(smem + C::OFF_SFW + stage * C::SF_BYTES,
+                          p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + static_cast<int64_t>(ks) * C::SF_ATOMS) * 512,
+                          atoms * 512, &wfull[stage]);
+            }
+            __syncwarp();
+            if (++stage == WS) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    } else if (warp == 1) {
+        // scale copies and MMAs: the whole warp runs the loop; one elected lane issues
+        int ws = 0, ts = 0;
+        uint32_t wph = 0, tph = 0;
+        bool ok = true;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&wfull[ws], wph, p.status, 52) || !mbar_wait_warp(&tready[ts], tph, p.status, 53)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // TMEM scale slot of this weight stage (free: its previous MMAs completed before the
+            // producer could refill the stage)
+            const uint32_t slot = tmem_base + C::SF_TMEM_BASE + ws * C::SLOT_COLS;
+            const uint32_t sfw_s = smem_u32(smem + C::OFF_SFW + ws * C::SF_BYTES);
+            const uint32_t sft_s = smem_u32(smem + C::OFF_SFT + ts * C::SF_BYTES);
+            const uint32_t w_s = smem_u32(smem + C::OFF_W + ws * C::W_BYTES);
+            const uint32_t t_s = smem_u32(smem + C::OFF_T + ts * C::T_BYTES);
+            if (elect_one()) {
+#pragma unroll
+                for (int a = 0; a < C::SF_ATOMS; ++a) {
+                    tc_cp_scales(slot + a * 4, smem_desc(sfw_s + a * 512, 0, 128, kLayoutNone));
+                    tc_cp_scales(slot + C::SF_ATOMS * 4 + a * 4, smem_desc(sft_s + a * 512, 0, 128, kLayoutNone));
+                }
+#pragma unroll
+                for (int j = 0; j < C::KSTEPS; ++j) {
+                    if (ks * C::BK + j * C::MMA_K < p.K) {
+                        const int kb = j * C::KB_PER_MMA;
+                        const int atom = kb >> 2;
+                        mma_block_scaled<KIND>(tmem_base, smem_desc(w_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               smem_desc(t_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               mma_idesc<KIND>(128, C::TOK, static_cast<uint32_t>(kb & 3)),
+                                               slot + atom * 4, slot + C::SF_ATOMS * 4 + atom * 4,
+                                               (ks > k0 || j > 0) ? 1u : 0u);
+                    }
+                }
+                tc_commit(&wempty[ws]);
+                tc_commit(&tempty[ts]);
+            }
+            __syncwarp();
+            if (++ws == WS) {
+                ws = 0;
+                wph ^= 1u;
+            }
+            if (++ts == TS) {
+                ts = 0;
+                tph ^= 1u;
+            }
+        }
+        if (ok && elect_one()) tc_commit(accf);
+        __syncwarp();
+    } else if (warp == 2) {
+        // token producer: the stage's bf16 rows, boxes of 64 elements (128 bytes) x 32 rows
+        const uint64_t pol = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&xempty[stage], phase ^ 1u, p.status, 54)) break;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&xfull[stage], C::X_BYTES);
+#pragma unroll
+                for (int b = 0; b < C::X_BOXES; ++b)
+                    tma_load_2d(&tma_x, &xfull[stage], smem + C::OFF_X + stage * C::X_BYTES + b * C::TOK * 128,
+                                (ks * C::BK + b * 64) * 2, 0, pol);
+            }
+            __syncwarp();
+            if (++stage == XS) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    } else {
+        // token quantizers: unit (row, j) = 32 elements; a warp takes the 32 token rows of one unit
+        // column, so its 16-byte reads of the swizzled rows fall in distinct banks
+        const int qt = (warp - 3) * 32 + lane;
+        constexpr int UPR = C::BK / 32;  // units per token row and stage (8 FP4, 4 MXFP8)
+        const bool active = qt < C::TOK * UPR;
+        const int row = qt & 31, j = qt >> 5;
+        float g_a = 1.0f;
+        if constexpr (KIND == 1) {
+            g_a = *p.g_a;
+            if (qt < 128) {
+                const float d = __fmul_rn(e4m3_decode_pos(static_cast<uint32_t>(qt)), g_a);
+                tab_d[qt] = d;
+                tab_r[qt] = __frcp_rn(d);  // fl(1/d), +inf for d = 0
+            }
+            named_barrier_sync(1, 32 * C::QWARPS);
+        }
+        int xs = 0, ts = 0;
+        uint32_t xph = 0, tph = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&xfull[xs], xph, p.status, 55) || !mbar_wait_warp(&tempty[ts], tph ^ 1u, p.status, 56))
+                break;
+            if (active && static_cast<int64_t>(ks) * C::BK + j * 32 < p.K) {
+                const uint32_t x_s = smem_u32(smem + C::OFF_X + xs * C::X_BYTES);
+                const uint32_t t_s = smem_u32(smem + C::OFF_T + ts * C::T_BYTES);
+                uint8_t* sft = smem + C::OFF_SFT + ts * C::SF_BYTES;
+                uint32_t w[16];
+                const uint32_t rb = x_s + (j >> 1) * C::TOK * 128 + row * 128;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 t = ld_shared_v4(rb + ((((j & 1) * 4 + i) ^ (row & 7)) << 4));
+                    w[4 * i] = t.x;
+                    w[4 * i + 1] = t.y;
+                    w[4 * i + 2] = t.z;
+                    w[4 * i + 3] = t.w;
+                }
+                uint32_t codes[8], seen = 0;
+                const uint32_t sc = quantize32<KIND, (QRULE < 0 ? 0 : QRULE), false>(w, g_a, tab_d, tab_r, codes, seen);
+                const uint32_t sw = static_cast<uint32_t>(row & 7);
+                const uint32_t t_row = t_s + row * 128;
+                // token scale atoms: the 32 token rows are rows 0-31 of a 128-row tile, byte row * 16 + block
+                if constexpr (KIND == 2) {  // MXFP8: 32 bytes of codes, one scale block
+                    st_shared_v4(t_row + (((2 * j) ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    st_shared_v4(t_row + (((2 * j + 1) ^ sw) << 4), make_uint4(codes[4], codes[5], codes[6], codes[7]));
+                    sft[(j >> 2) * 512 + row * 16 + (j & 3)] = static_cast<uint8_t>(sc);
+                } else if constexpr (KIND == 1) {  // NVFP4: 16 bytes of codes, scale blocks 2j and 2j + 1
+                    st_shared_v4(t_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    *reinterpret_cast<uint16_t*>(sft + ((2 * j) >> 2) * 512 + row * 16 + ((2 * j) & 3)) =
+                        static_cast<uint16_t>(sc);
+                } else {  // MXFP4: 16 bytes of codes, one scale block
+                    st_shared_v4(t_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    sft[(j >> 2) * 512 + row * 16 + (j & 3)] = static_cast<uint8_t>(sc);
+                }
+            }
+            fence_proxy_async_smem();  // the token tile is read next by the tensor core
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&tready[ts]);
+                mbar_arrive(&xempty[xs]);
+            }
+            if (++xs == XS) {
+                xs = 0;
+                xph ^= 1u;
+            }
+            if (++ts == TS) {
+                ts = 0;
+                tph ^= 1u;
+            }
+        }
+    }
+
+    // reduction and epilogue: warp w of 3-10 holds the 16 tokens [16 h, +16) (h = (w - 3) / 4) of the
+    // 32 weight rows in its TMEM sub-partition.  The non-leaders send their partials to the leader's
+    // buffer ([split - 1][token quad][128 rows][4] fp32: a warp's 16-byte stores cover 512
+    // contiguous bytes) as soon as their MMAs are done; the leader adds them in split order.
+    const bool epi = warp >= 3;
+    const int sub = warp & 3;
+    const int h = (warp - 3) >> 2;
+    const int wrow = sub * 32 + lane;  // weight row within the tile
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    float acc[16];
+    cluster_wait();  // every CTA of the cluster has initialised its barriers
+    if (epi) {
+        const bool ok = mbar_wait(accf, 0, p.status, 57);
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(16 * h), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = ok ? __uint_as_float(r[i]) : 0.0f;
+        tc_fence_before();
+    }
+    if (epi && split != 0) {
+        const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow) * 4), 0);
+        const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            st_async_v4(dst + q * 128 * 16, acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3], bar);
+    }
+    if (epi && split == 0) {
+        const bool got = mbar_wait(rfull, 0, p.status, 58);
+        for (uint32_t sp = 1; got && sp < splits; ++sp) {
+            const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = src[q * 128];
+                acc[4 * q] = __fadd_rn(acc[4 * q], v.x);
+                acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
+                acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
+                acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+            }
+        }
+        const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
+        const int n = nt * 128 + wrow;
+        if (n < p.N) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int m = 16 * h + i;
+                if (m < p.M) {
+                    const float v = KIND == 1 ? __fmul_rn(acc[i], alpha) : acc[i];
+                    if constexpr (OUT_F32) {
+                        static_cast<float*>(p.out)[static_cast<int64_t>(m) * p.N + n] = v;
+                    } else {
+                        static_cast<__nv_bfloat16*>(p.out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(v);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ small-N linear kernel
+//
+// Linear layers with few output columns (N <= 128, e.g. a fused N = 96 projection) and many
+// tokens.  With one column tile the GEMM reads every activation row exactly once, so it quantizes
+// the bf16 rows itself instead of reading codes that a separate quantizer pass wrote: A crosses
+// HBM once, as bf16, and no codes round-trip through it.  One CTA per 128-row M tile and K split;
+// the S CTAs of a cluster split the K stages and reduce their partial accumulators through
+// distributed shared memory in the leader, as the split-K kernel does.
+//   warp 0      TMA producer: the stage's bf16 rows (boxes of 64 elements x 128 rows, 128B
+//               swizzle), the weight codes (128 rows x 128 bytes) and the weight scale tiles
+//   warp 1      TMEM owner; copies the stage's scale tiles into TMEM (tcgen05.cp) and issues the MMAs
+//   warps 2-17  quantize the stage's rows into the A tile (codes in the 128B-swizzled operand
+//               layout, scales in the 512-byte tile layout) with the streaming quantizer's
+//               arithmetic; after the last stage they are the epilogue.  The quantization is
+//               latency-bound per warp, so it gets 16 warps (8 held the kernel to about 18 GB/s of
+//               bf16 rows per SM).
+template <int KIND>
+struct RowqCfg {
+    static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
+    static constexpr int BK = 128 * EPB;          // K elements per stage: 128 code bytes per row
+    static constexpr int KSTEPS = BK / MMA_K;     // 4 MMAs per stage
+    static constexpr int KB_PER_MMA = MMA_K / BS;
+    static constexpr int SF_ATOMS = BK / BS / 4;  // 512-byte scale tiles per 128 rows per stage
+    static constexpr int BN = 128;
+    static constexpr int STAGES = (KIND == 2) ? 3 : 2;
+    static constexpr int X_BOXES = BK / 64;       // bf16 boxes of 64 elements x 128 rows
+    static constexpr int X_BYTES = X_BOXES * 128 * 128;
+    static constexpr int A_BYTES = 128 * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SF_BYTES = SF_ATOMS * 512;
+    static constexpr int QWARPS = 16;
+    static constexpr int THREADS = (2 + QWARPS) * 32;
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_A = OFF_X + STAGES * X_BYTES;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SF_BYTES;
+    static constexpr int OFF_TAB = OFF_SFB + STAGES * SF_BYTES;  // NVFP4 d and 1/d per scale code
+    static constexpr int OFF_BAR = OFF_TAB + 1024;
+    static constexpr int N_BARS = 3 * STAGES + 3;  // full, qready, empty per stage; accf, rready, rfull
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
+    static constexpr int SF_COLS_STAGE = 2 * SF_ATOMS * 4;  // A then B scale tiles, 4 columns each
+    static constexpr int SF_TMEM_BASE = BN;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static_assert(KSTEPS == 4, "4 MMAs per stage");
+    static_assert(SF_TMEM_BASE + STAGES * SF_COLS_STAGE <= static_cast<int>(TMEM_COLS), "TMEM budget");
+    static_assert((kMaxSplits - 1) * 128 * BN * 4 <= OFF_TAB, "reduction buffer inside the ring");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int KIND, bool OUT_F32, int QRULE>
+__global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
+    gemm_rowq_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_b,
+                     const GemmArgs p) {
+    using C = RowqCfg<KIND>;
+    constexpr int STAGES = C::STAGES, BN = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* qready = full + STAGES;
+    uint64_t* empty = qready + STAGES;
+    uint64_t* accf = empty + STAGES;
+    uint64_t* rready = accf + 1;  // non-leaders: the leader's ring is free for the partials
+    uint64_t* rfull = accf + 2;   // leader: every partial has landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
+    float* tab_d = reinterpret_cast<float*>(smem + C::OFF_TAB);
+    float* tab_r = tab_d + 128;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t split = cluster_ctarank();
+    const uint32_t splits = p.k_split;
+    const int mt = static_cast<int>(blockIdx.x / splits);
+    const int mrows = min(128, p.M - mt * 128);  // valid rows of this M tile
+    const int per = (p.k_stages + static_cast<int>(splits) - 1) / static_cast<int>(splits);
+    const int k0 = static_cast<int>(split) * per;
+    const int k1 = min(p.k_stages, k0 + per);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tma_x);
+        prefetch_tmap(&tma_b);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&qready[s], C::QWARPS);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(rready, 1);
+        mbar_init(rfull, 1);
+        if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * static_cast<uint32_t>(mrows) * BN * 4);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_arrive_relaxed();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_launch_dependents();  // the next kernel on the stream may start its prologue
+
+    if (warp == 0) {
+        // TMA producer: the whole warp runs the loop; one elected lane issues
+        const uint64_t pol_x = policy_evict_first();
+        const uint64_t pol_b = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 41)) break;
+            if (elect_one()) {
+                const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
+                mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::B_BYTES + atoms * 512);
+#pragma unroll
+                for (int b = 0; b < C::X_BOXES; ++b)
+                    tma_load_2d(&tma_x, &full[stage], smem + C::OFF_X + stage * C::X_BYTES + b * 128 * 128,
+                                (ks * C::BK + b * 64) * 2, mt * 128, pol_x);
+                tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, 0, pol_b);
+                bulk_load(smem + C::OFF_SFB + stage * C::SF_BYTES,
+                          p.b_sf + static_cast<int64_t>(ks) * C::SF_ATOMS * 512, atoms * 512, &full[stage]);
+            }
+            __syncwarp();
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    } else if (warp == 1) {
+        // scale copies and MMAs: the whole warp runs the loop; one elected lane issues
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&full[stage], phase, p.status, 42) ||
+                !mbar_wait_warp(&qready[stage], phase, p.status, 43)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
+            const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SF_BYTES);
+            const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SF_BYTES);
+            const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+            const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+            if (elect_one()) {
+#pragma unroll
+                for (int a = 0; a < C::SF_ATOMS; ++a) {
+                    tc_cp_scales(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
+                    tc_cp_scales(sf_col + C::SF_ATOMS * 4 + a * 4, smem_desc(sfb_s + a * 512, 0, 128, kLayoutNone));
+                }
+#pragma unroll
+                for (int j = 0; j < C::KSTEPS; ++j) {
+                    if (ks * C::BK + j * C::MMA_K < p.K) {
+                        const int kb = j * C::KB_PER_MMA;
+                        const int atom = kb >> 2;
+                        mma_block_scaled<KIND>(tmem_base, smem_desc(a_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               smem_desc(b_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                               mma_idesc<KIND>(kBM, BN, static_cast<uint32_t>(kb & 3)),
+                                               sf_col + atom * 4, sf_col + C::SF_ATOMS * 4 + atom * 4,
+                                               (ks > k0 || j > 0) ? 1u : 0u);
+                    }
+                }
+                tc_commit(&empty[stage]);
+            }
+            __syncwarp();
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (ok && elect_one()) tc_commit(accf);
+        __syncwarp();
+    } else {
+        // quantizers: thread qt takes units (row, j) of 32 elements, a warp 32 consecutive rows of
+        // one unit column, so its 16-byte reads of the swizzled bf16 rows fall in distinct banks
+        static_assert(128 * (C::BK / 32) % (32 * C::QWARPS) == 0, "whole units per thread");
+        const int qt = (warp - 2) * 32 + lane;
+        constexpr int UPR = C::BK / 32;                 // units per row and stage
+        constexpr int UPT = 128 * UPR / (32 * C::QWARPS);  // units per thread and stage
+        float g_a = 1.0f;
+        if constexpr (KIND == 1) {
+            g_a = *p.g_a;
+            if (qt < 128) {
+                const float d = __fmul_rn(e4m3_decode_pos(static_cast<uint32_t>(qt)), g_a);
+                tab_d[qt] = d;
+                tab_r[qt] = __frcp_rn(d);  // fl(1/d), +inf for d = 0
+            }
+            named_barrier_sync(1, 32 * C::QWARPS);
+        }
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            if (!mbar_wait_warp(&full[stage], phase, p.status, 44)) break;
+            const uint32_t x_s = smem_u32(smem + C::OFF_X + stage * C::X_BYTES);
+            const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+            uint8_t* sfa = smem + C::OFF_SFA + stage * C::SF_BYTES;
+#pragma unroll
+            for (int u = 0; u < UPT; ++u) {
+                const int v = qt + u * 32 * C::QWARPS;
+                const int row = v & 127, j = v >> 7;
+                if (static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
+                uint32_t w[16];
+                const uint32_t rb = x_s + (j >> 1) * 128 * 128 + row * 128;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 t = ld_shared_v4(rb + ((((j & 1) * 4 + i) ^ (row & 7)) << 4));
+                    w[4 * i] = t.x;
+                    w[4 * i + 1] = t.y;
+                    w[4 * i + 2] = t.z;
+                    w[4 * i + 3] = t.w;
+                }
+                uint32_t codes[8], seen = 0;
+                const uint32_t sc = quantize32<KIND, (QRULE < 0 ? 0 : QRULE), false>(w, g_a, tab_d, tab_r, codes, seen);
+                const uint32_t sw = static_cast<uint32_t>(row & 7);
+                const uint32_t sf_row = (row & 31) * 16 + ((row >> 5) & 3) * 4;
+                const uint32_t a_row = a_s + row * 128;
+                if constexpr (KIND == 2) {  // MXFP8: 32 bytes of codes, one scale block
+                    st_shared_v4(a_row + (((2 * j) ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    st_shared_v4(a_row + (((2 * j + 1) ^ sw) << 4), make_uint4(codes[4], codes[5], codes[6], codes[7]));
+                    sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
+                } else if constexpr (KIND == 1) {  // NVFP4: 16 bytes of codes, scale blocks 2j and 2j + 1
+                    st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    *reinterpret_cast<uint16_t*>(sfa + ((2 * j) >> 2) * 512 + sf_row + ((2 * j) & 3)) =
+                        static_cast<uint16_t>(sc);
+                } else {  // MXFP4: 16 bytes of codes, one scale block
+                    st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+                    sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
+                }
+            }
+            fence_proxy_async_smem();  // the A tile and scale tiles are read next by the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qready[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+
+    // reduction and epilogue: warps 2-17 hold 32 accumulator columns of one TMEM sub-partition each;
+    // the leader frees its ring for the partials once its MMAs are done, the others send their
+    // valid rows with st.async (column-quad-major layout, as in the split-K kernel) and leave
+    constexpr int COLS = BN / (C::QWARPS / 4);
+    const bool epi = warp >= 2;
+    const int sub = warp & 3;
+    const int col0 = ((warp - 2) >> 2) * COLS;
+    const int row = sub * 32 + lane;
+    float* red = reinterpret_cast<float*>(smem);
+    float acc[COLS];
+    cluster_wait();  // every CTA of the cluster has initialised its barriers
+    if (epi) {
+        const bool ok = mbar_wait(accf, 0, p.status, 45);
+        if (split == 0 && warp == 2 && lane == 0)
+            for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
+#pragma unroll
+        for (int c = 0; c < COLS / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c * 32 + i] = ok ? __uint_as_float(r[i]) : 0.0f;
+        }
+        tc_fence_before();
+    }
+    if (epi && split != 0 && row < mrows && mbar_wait_cluster(rready, 0, p.status, 46)) {
+        const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (BN / 4) + col0 / 4) * 128 + row) * 4), 0);
+        const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
+#pragma unroll
+        for (int v = 0; v < COLS / 4; ++v)
+            st_async_v4(dst + v * 128 * 16, acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3], bar);
+    }
+    if (epi && split == 0 && row < mrows) {
+        const bool got = mbar_wait(rfull, 0, p.status, 47);
+        for (uint32_t sp = 1; got && sp < splits; ++sp) {
+            const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (BN / 4) + col0 / 4) * 128 + row;
+#pragma unroll
+            for (int v = 0; v < COLS / 4; ++v) {
+                const float4 q = src[v * 128];
+                acc[4 * v] = __fadd_rn(acc[4 * v], q.x);
+                acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], q.y);
+                acc[4 * v + 2] = __fadd_rn(acc[4 * v + 2], q.z);
+                acc[4 * v + 3] = __fadd_rn(acc[4 * v + 3], q.w);
+            }
+        }
+        const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
+        const int64_t m = static_cast<int64_t>(mt) * 128 + row;
+        if constexpr (!OUT_F32) {
+            uint16_t* o16 = reinterpret_cast<uint16_t*>(p.out) + m * p.N;
+#pragma unroll
+            for (int i = 0; i < COLS / 2; ++i) {
+                const float lo = KIND == 1 ? __fmul_rn(acc[2 * i], alpha) : acc[2 * i];
+                const float hi = KIND == 1 ? __fmul_rn(acc[2 * i + 1], alpha) : acc[2 * i + 1];
+                const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+                const uint32_t pk = *reinterpret_cast<const uint32_t*>(&b);
+                const int n = col0 + 2 * i;
+                if (n < p.N) o16[n] = static_cast<uint16_t>(pk & 0xFFFFu);
+                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(pk >> 16);
+            }
+        } else {
+            float* orow = static_cast<float*>(p.out) + m * p.N;
+#pragma unroll
+            for (int i = 0; i < COLS; ++i)
+                if (col0 + i < p.N) orow[col0 + i] = __fmul_rn(acc[i], alpha);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ CTA-pair kernel
 //
 // Two CTAs of a cluster on two SMs compute one 256 x BN tile with cta_group::2 MMAs: CTA r loads
@@ -1327,6 +1984,97 @@ int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cuda
     return MXQ_OK;
 }
 
+template <int KIND, bool F32, int QRULE>
+int run_decode(const void* x, const void* B_q, GemmArgs args, int splits, cudaStream_t stream) {
+    using C = DecCfg<KIND>;
+    auto kern = gemm_decode_kernel<KIND, F32, QRULE>;
+    CUtensorMap tx, tw;
+    // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 32 rows; W codes 128 rows x 128 bytes
+    if (!make_map(&tx, x, 2 * static_cast<uint64_t>(args.K), args.M, C::TOK) ||
+        !make_map(&tw, B_q, args.K / C::EPB, args.N, 128))
+        return MXQ_ERR_CUDA;
+    args.m_tiles = 1;
+    args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
+    args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
+    args.k_split = static_cast<uint32_t>(splits);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(args.n_tiles * splits);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tw, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
+template <int KIND, bool F32, int QRULE>
+int run_rowq(const void* x, const void* B_q, GemmArgs args, int splits, cudaStream_t stream) {
+    using C = RowqCfg<KIND>;
+    auto kern = gemm_rowq_kernel<KIND, F32, QRULE>;
+    CUtensorMap tx, tb;
+    // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 128 rows; W codes as the GEMM's
+    if (!make_map(&tx, x, 2 * static_cast<uint64_t>(args.K), args.M, 128) ||
+        !make_map(&tb, B_q, args.K / C::EPB, args.N, 128))
+        return MXQ_ERR_CUDA;
+    args.m_tiles = static_cast<int>(ceil_div(args.M, 128));
+    args.n_tiles = 1;
+    args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
+    args.k_split = static_cast<uint32_t>(splits);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static bool attr_done[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(args.m_tiles * splits);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    return MXQ_OK;
+}
+
+// K splits of the small-N kernel: as many as keep all M tiles' clusters resident at once (at most
+// 4), each split owning at least one K stage.
+int rowq_splits(int64_t M, int64_t K, int bk) {
+    const int64_t m_tiles = ceil_div(M, 128);
+    const int64_t k_stages = ceil_div(K, bk);
+    int64_t s = sm_count() / m_tiles;
+    if (s > static_cast<int64_t>(kMaxSplits)) s = kMaxSplits;
+    if (s > k_stages) s = k_stages;
+    if (s < 2) return 1;
+    const int64_t per = ceil_div(k_stages, s);
+    return static_cast<int>(ceil_div(k_stages, per));
+}
+
 // K splits for a one-row-tile problem: as many as keep every cluster of the grid resident at once
 // (at most 4), each split owning at least one K stage.
 int splitk_count(int64_t N, int64_t K, int bk) {
@@ -1390,12 +2138,22 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
 namespace {
 template <int KIND, bool F32>
 int fused_rule(const void* W_q, const GemmArgs& a, int rule, int splits, cudaStream_t stream) {
-    return rule == MXQ_RULE_CEIL ? run_splitk<KIND, F32, MXQ_RULE_CEIL>(nullptr, W_q, a, splits, stream, true)
-                                 : run_splitk<KIND, F32, MXQ_RULE_EVEN>(nullptr, W_q, a, splits, stream, true);
+    return rule == MXQ_RULE_CEIL ? run_decode<KIND, F32, MXQ_RULE_CEIL>(a.x, W_q, a, splits, stream)
+                                 : run_decode<KIND, F32, MXQ_RULE_EVEN>(a.x, W_q, a, splits, stream);
 }
+template <int KIND, bool F32>
+int rowq_rule(const void* x, const void* W_q, const GemmArgs& a, int rule, int splits, cudaStream_t stream) {
+    return rule == MXQ_RULE_CEIL ? run_rowq<KIND, F32, MXQ_RULE_CEIL>(x, W_q, a, splits, stream)
+                                 : run_rowq<KIND, F32, MXQ_RULE_EVEN>(x, W_q, a, splits, stream);
+}
+
+// Few output columns and more tokens than the split-K kernel quantizes itself: one column tile, so
+// the small-N kernel reads each activation row once and quantizes it on the way in.
+bool rowq_applies(int64_t M, int64_t N) { return M > 32 && N <= RowqCfg<0>::BN; }
 }  // namespace
 
 int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt) {
+    if (rowq_applies(M, N)) return rowq_splits(M, K, fmt == MXQ_MXFP8 ? RowqCfg<2>::BK : RowqCfg<0>::BK);
     // the bf16 activations of a stage (rows rounded up to 8, BK elements) must fit the A buffer
     if (M > 32) return 0;
     const int bk = fmt == MXQ_MXFP8 ? Cfg<2, 128, 6>::BK : Cfg<0, 128, 6>::BK;
@@ -1407,7 +2165,8 @@ int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, con
                         int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,
                         cudaStream_t stream) {
     const int splits = linear_fused_splits(M, N, K, fmt);
-    if (splits < 2) return kNotFused;
+    const bool rowq = rowq_applies(M, N);
+    if (!rowq && splits < 2) return kNotFused;
     GemmArgs a = {};
     a.x = x;
     a.b_sf = W_sf;
@@ -1421,6 +2180,18 @@ int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, con
     a.b_row_tiles = static_cast<int>(ceil_div(N, 128));
     a.status = status_ptr();
     const bool f32 = out_type == MXQ_OUT_FP32;
+    if (rowq) {
+        switch (fmt) {
+            case MXQ_MXFP4:
+                return f32 ? rowq_rule<0, true>(x, W_q, a, rule, splits, stream)
+                           : rowq_rule<0, false>(x, W_q, a, rule, splits, stream);
+            case MXQ_NVFP4:
+                return f32 ? run_rowq<1, true, 0>(x, W_q, a, splits, stream) : run_rowq<1, false, 0>(x, W_q, a, splits, stream);
+            default:
+                return f32 ? rowq_rule<2, true>(x, W_q, a, rule, splits, stream)
+                           : rowq_rule<2, false>(x, W_q, a, rule, splits, stream);
+        }
+    }
     switch (fmt) {
         case MXQ_MXFP4:
             return f32 ? fused_rule<0, true>(W_q, a, rule, splits, stream) : fused_rule<0, false>(W_q, a, rule, splits, stream);

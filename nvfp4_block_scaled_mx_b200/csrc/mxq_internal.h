@@ -65,12 +65,15 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
                 const float* g_B, int64_t M, int64_t N, int64_t K, int fmt, int out_type, void* out,
                 cudaStream_t stream, bool pdl_secondary);
 
-// Few-token linear layer in one launch: the split-K GEMM quantizes the bf16 activations x itself
-// (rule `rule` for MX formats, global scale g_A for NVFP4) with the quantizer's arithmetic, so the
-// result equals quantize-then-GEMM bit for bit.  Returns kNotFused (nothing launched) unless the
-// problem takes the split-K kernel with M <= 32 (several K splits); arguments already validated.
+// Linear layer in one launch where the GEMM quantizes the bf16 activations x itself (rule `rule`
+// for MX formats, global scale g_A for NVFP4) with the quantizer's arithmetic: the split-K GEMM for
+// up to 32 tokens with several K splits (the result equals quantize-then-GEMM bit for bit), and the
+// small-N kernel for more tokens and N <= 128.  Returns kNotFused (nothing launched) otherwise;
+// arguments already validated.
 constexpr int kNotFused = 1;
-// K splits of the one-launch path for this problem on the current device, 0 when it does not apply.
+// K splits of the one-launch path for this problem on the current device (the split-K GEMM
+// quantizing up to 32 token rows, or the small-N kernel quantizing whole 128-row M tiles for N <= 128;
+// 1 when that kernel runs without a K split), 0 when no one-launch path applies.
 int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt);
 int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
                         int64_t M, int64_t N, int64_t K, int fmt, int rule, int out_type, void* out,

@@ -104,3 +104,22 @@ def test_noalloc_writes_inside_its_output(fmt, M, N, K):
     expect = mxq.linear(A, Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=torch.bfloat16, g_W=g_w, g_A=g_a)
     torch.cuda.synchronize()
     assert torch.equal(o.t.view(torch.int16), expect.view(torch.int16))
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("M,N,K", [(33, 1, 64), (129, 96, 1024), (300, 17, 576)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_small_n_linear_writes_inside_its_output(fmt, M, N, K, out_dtype):
+    """The small-N linear kernel (more than 32 tokens, N <= 128) stores row by row with N tails."""
+    A = synth.random_bf16((M, K), 13 * M + K, device="cuda")
+    W = synth.random_bf16((N, K), 17 * N + K, std=0.02, device="cuda")
+    g_a = g_w = None
+    if fmt == "nvfp4":
+        g_a, g_w = mxq.global_scale(A)[0], mxq.global_scale(W)[0]
+    Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w)
+    es = 4 if out_dtype == torch.float32 else 2
+    o = Canary(M * N * es, out_dtype, (M, N))
+    mxq.linear(A, Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=out_dtype, g_W=g_w, g_A=g_a, out=o.t)
+    torch.cuda.synchronize()
+    assert o.intact(), "small-N linear output written outside its buffer"
+    assert mxq.mxq_device_status(reset=True) == 0

@@ -164,6 +164,40 @@ def test_linear_one_launch_equals_quantize_then_gemm(fmt, rule, M, N, K):
     assert mxq.mxq_device_status(reset=True) == 0
 
 
+@pytest.mark.parametrize("fmt,rule", [("mxfp4", "ceil"), ("mxfp4", "even"), ("nvfp4", "even"), ("mxfp8", "even"),
+                                      ("mxfp8", "ceil")])
+@pytest.mark.parametrize("M,N,K", [(33, 96, 512), (129, 1, 640), (300, 128, 320), (1000, 100, 1024), (257, 17, 5120),
+                                   (4000, 96, 256)])
+def test_linear_small_n_matches_oracle(fmt, rule, M, N, K):
+    """More than 32 tokens and N <= 128: mxq_linear is one launch, the small-N kernel quantizing each
+    128-row activation tile on its way into the tensor cores (K split over a cluster).  Checked
+    against the oracle from the bf16 inputs, fp32 and bf16 out, with ragged M tiles, N = 1 and
+    N < 128 column tails, a K tail that leaves the last stage partly empty (K = 320) and one K
+    stage only (K = 256 for FP4: no split)."""
+    if fmt == "mxfp8" and K % 32:
+        pytest.skip("K")
+    assert mxq.linear_kernel_count(M, N, K, fmt) == 1
+    A = synth.random_bf16((M, K), 31 + M + K, std=1.0)
+    W = synth.random_bf16((N, K), 37 + N, std=0.02)
+    a, w = _quant_pair(A, W, fmt, rule, "even")
+    ref, abs_sum = oracle.gemm(a[0], a[1], w[0], w[1], M, N, K, FMTS[fmt], gA=a[2], gB=w[2])
+    Wd, Ad = W.cuda(), A.cuda()
+    g_w = g_a = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(Wd)
+        g_a, _ = mxq.global_scale(Ad)
+    Wq, Wsf = mxq.quantize(Wd, fmt, "even", global_scale=g_w)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out = mxq.linear(Ad, Wq, Wsf, N, fmt, act_rule=rule, out_dtype=out_dtype, g_W=g_w, g_A=g_a)
+        torch.cuda.synchronize()
+        gpu = out.double().cpu().numpy()
+        if out_dtype == torch.float32:
+            check_fp32(gpu, ref, abs_sum, "small-N linear %s %s" % (fmt, (M, N, K)))
+        else:
+            check_bf16(gpu, ref, abs_sum, "small-N linear %s %s" % (fmt, (M, N, K)))
+    assert mxq.mxq_device_status(reset=True) == 0
+
+
 def test_linear_kernel_count():
     """mxq_linear_kernel_count reports the one-launch path exactly where the bit-equality test above
     exercises it: up to 32 tokens with several K splits."""
@@ -173,6 +207,8 @@ def test_linear_kernel_count():
     assert mxq.linear_kernel_count(100, 300, 320, "mxfp4") == 2
     assert mxq.linear_kernel_count(8192, 34816, 5120, "mxfp4") == 2
     assert mxq.linear_kernel_count(32, 34816, 5120, "mxfp4") == 2  # one K split: quantizer + GEMM
+    assert mxq.linear_kernel_count(8192, 96, 5120, "mxfp8") == 1  # small N: the GEMM quantizes its rows
+    assert mxq.linear_kernel_count(8192, 129, 5120, "mxfp8") == 2
 
 
 def test_tiny_config_full():
