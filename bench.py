@@ -252,6 +252,31 @@ def run_mxq(args, world, rank, local):
     torch.cuda.synchronize()
     mxq.mxq_device_status(reset=True)
 
+    timing = "eager calls through the binding"
+    if M <= 32:
+        # few tokens: a call is a few microseconds of GPU work, less than the host needs to launch it
+        # through the Python binding (about 12 us), so each step replays a CUDA graph holding that
+        # step's call (one graph per weight copy), as serving replays its decode steps; the host's
+        # launch cost stays outside the measurement
+        gs = torch.cuda.Stream(device=dev)
+        graphs = []
+        torch.cuda.synchronize()
+        for wq, wsf in wset:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gs):
+                mxq.linear(A, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
+                           workspace=ws, out=out)
+            graphs.append(g)
+
+        def step():
+            graphs[it[0] % copies].replay()
+            it[0] += 1
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        timing = "one CUDA graph replay per step (the host launch cost is outside the graph)"
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
@@ -353,7 +378,7 @@ def run_mxq(args, world, rank, local):
            "scaling": "weak", "vs_baseline": None, "dtype": "e2m1xe2m1->f32 (bf16 out)" if fmt != "mxfp8" else
            "e4m3xe4m3->f32 (bf16 out)", "data": "synthetic (seeded, random-init weights)",
            "config": {"workload": workload, "M": M, "N": N, "K": K, "fmt": fmt, "act_rule": cfg["a_rule"],
-                      "weight_rule": cfg["w_rule"], "out": cfg["out"], "l2": l2_note,
+                      "weight_rule": cfg["w_rule"], "out": cfg["out"], "l2": l2_note, "timing": timing,
                       "parallelism": "replicas x%d (no collective)" % world},
            "gpu_launches": mxq.linear_kernel_count(M, N, K, fmt) * args.steps, "roofline": roofline, "quantize": quant, "quantize_weight": quant_w,
            "fake_quantize": fake_quant,
@@ -403,6 +428,15 @@ def other_workloads(stream, bf16_tflops):
             del q, sf, flush
         for _ in range(3):
             f()
+        if M <= 32:  # few tokens: replay a graph of the call, as for the decode bench (host launch cost outside)
+            gs = torch.cuda.Stream()
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=gs):
+                mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], g_W=g_w, g_A=g_a, workspace=ws, out=out)
+            f = gr.replay
+            for _ in range(3):
+                f()
         iters = 200 if M * N < 1e8 else 30
         t = time_loop(f, iters, stream)
         peak = bf16_tflops * (FP8_PER_BF16 if fmt == "mxfp8" else FP4_PER_BF16)
@@ -411,7 +445,8 @@ def other_workloads(stream, bf16_tflops):
         if name == "decode":  # weight-stream bound: codes + scales of W per call
             wbytes = W_q.numel() + W_sf.numel()
             r["weight_gbs"] = round(wbytes / t / 1e9, 1)
-            r["l2"] = "back-to-back calls on one weight copy (L2-resident); --workload decode streams them from HBM"
+            r["l2"] = ("back-to-back CUDA graph replays of the call on one weight copy (L2-resident); --workload decode "
+                       "streams them from HBM")
         r.update(qr)
         res[name] = r
         del A, W_q, W_sf, ws, out

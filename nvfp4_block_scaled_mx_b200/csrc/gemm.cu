@@ -802,7 +802,9 @@ struct DecCfg {
     static constexpr int KB_PER_MMA = MMA_K / BS;
     static constexpr int SF_ATOMS = BK / BS / 4;
     static constexpr int TOK = 32;                   // MMA N: token rows (rows >= M are zero)
-    static constexpr int WSTAGES = 5, XSTAGES = 3, TSTAGES = 6;
+    // a deep weight ring: about 112 KB per SM in flight is what the HBM latency under this load
+    // needs (with 5 stages the first stage of every CTA arrived only after about 2.3 us)
+    static constexpr int WSTAGES = (KIND == 1) ? 6 : 7, XSTAGES = 2, TSTAGES = 5;
     static constexpr int W_BYTES = 128 * 128;
     static constexpr int SF_BYTES = SF_ATOMS * 512;
     static constexpr int X_BOXES = BK / 64;
@@ -828,13 +830,14 @@ struct DecCfg {
     static_assert(KSTEPS == 4, "4 MMAs per stage");
     static_assert(SF_TMEM_BASE + WSTAGES * SLOT_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
     static_assert(OFF_W % 1024 == 0 && OFF_X % 1024 == 0 && OFF_T % 1024 == 0, "swizzled buffers 1024-aligned");
+    static_assert(TOK * 128 * 2 <= XSTAGES * X_BYTES, "output staging tile inside the token ring");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int KIND, bool OUT_F32, int QRULE>
 __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_w,
-                       const GemmArgs p) {
+                       const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
     using C = DecCfg<KIND>;
     constexpr int WS = C::WSTAGES, XS = C::XSTAGES, TS = C::TSTAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -1097,7 +1100,24 @@ __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
         }
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
         const int n = nt * 128 + wrow;
-        if (n < p.N) {
+        if (!OUT_F32 && p.tma_store) {
+            // the [32 tokens][128 columns] bf16 tile through shared memory (the token ring is idle now:
+            // every stage has been quantized) and one TMA store, clipped at the M and N edges; direct
+            // stores would write one 2-byte element per token row and lane
+            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::OFF_X);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float v = KIND == 1 ? __fmul_rn(acc[i], alpha) : acc[i];
+                stg[(16 * h + i) * 128 + wrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
+            fence_proxy_async_smem();
+            named_barrier_sync(2, 32 * C::QWARPS);
+            if (warp == 3 && lane == 0) {
+                tma_store_2d(&tma_out, stg, nt * 128, 0);
+                bulk_commit_group();
+                bulk_wait_group0();
+            }
+        } else if (n < p.N) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int m = 16 * h + i;
@@ -1126,15 +1146,16 @@ __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
 // the bf16 rows itself instead of reading codes that a separate quantizer pass wrote: A crosses
 // HBM once, as bf16, and no codes round-trip through it.  One CTA per 128-row M tile and K split;
 // the S CTAs of a cluster split the K stages and reduce their partial accumulators through
-// distributed shared memory in the leader, as the split-K kernel does.
-//   warp 0      TMA producer: the stage's bf16 rows (boxes of 64 elements x 128 rows, 128B
-//               swizzle), the weight codes (128 rows x 128 bytes) and the weight scale tiles
-//   warp 1      TMEM owner; copies the stage's scale tiles into TMEM (tcgen05.cp) and issues the MMAs
-//   warps 2-17  quantize the stage's rows into the A tile (codes in the 128B-swizzled operand
-//               layout, scales in the 512-byte tile layout) with the streaming quantizer's
-//               arithmetic; after the last stage they are the epilogue.  The quantization is
-//               latency-bound per warp, so it gets 16 warps (8 held the kernel to about 18 GB/s of
-//               bf16 rows per SM).
+// distributed shared memory in the leader, as the split-K kernel does.  The bf16 rows stream
+// through a ring of 16 KB slots (64 elements x 128 rows, 128B swizzle) deeper than the stages the
+// tensor cores consume, so that about 128 KB per SM stay in flight from HBM.
+//   warp 0       TMA producer of the bf16 slots
+//   warp 1       TMEM owner; copies the stage's scale tiles into TMEM (tcgen05.cp), issues the MMAs
+//   warp 2       TMA producer of the weight stages (codes 128 rows x 128 bytes, scale tiles)
+//   warps 3-18   quantize each stage's rows into the A tile (codes in the 128B-swizzled operand
+//                layout, scales in the 512-byte tile layout) with the streaming quantizer's
+//                arithmetic (16 warps: the quantization is latency-bound per warp); after the last
+//                stage they are the epilogue, which stores through shared memory and TMA
 template <int KIND>
 struct RowqCfg {
     static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
@@ -1143,46 +1164,53 @@ struct RowqCfg {
     static constexpr int KB_PER_MMA = MMA_K / BS;
     static constexpr int SF_ATOMS = BK / BS / 4;  // 512-byte scale tiles per 128 rows per stage
     static constexpr int BN = 128;
-    static constexpr int STAGES = (KIND == 2) ? 3 : 2;
-    static constexpr int X_BOXES = BK / 64;       // bf16 boxes of 64 elements x 128 rows
-    static constexpr int X_BYTES = X_BOXES * 128 * 128;
+    static constexpr int XSLOTS = 8;              // bf16 slots of 64 elements x 128 rows
+    static constexpr int XPS = BK / 64;           // slots per stage (4 FP4, 2 MXFP8)
+    static constexpr int ASTAGES = 2, BSTAGES = 2;
+    static constexpr int X_BYTES = 128 * 128;
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int SF_BYTES = SF_ATOMS * 512;
     static constexpr int QWARPS = 16;
-    static constexpr int THREADS = (2 + QWARPS) * 32;
+    static constexpr int THREADS = (3 + QWARPS) * 32;
     static constexpr int OFF_X = 0;
-    static constexpr int OFF_A = OFF_X + STAGES * X_BYTES;
-    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + STAGES * SF_BYTES;
-    static constexpr int OFF_TAB = OFF_SFB + STAGES * SF_BYTES;  // NVFP4 d and 1/d per scale code
+    static constexpr int OFF_A = OFF_X + XSLOTS * X_BYTES;
+    static constexpr int OFF_B = OFF_A + ASTAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + BSTAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + ASTAGES * SF_BYTES;
+    static constexpr int OFF_TAB = OFF_SFB + BSTAGES * SF_BYTES;  // NVFP4 d and 1/d per scale code
     static constexpr int OFF_BAR = OFF_TAB + 1024;
-    static constexpr int N_BARS = 3 * STAGES + 3;  // full, qready, empty per stage; accf, rready, rfull
+    static constexpr int N_BARS = 2 * (XSLOTS + ASTAGES + BSTAGES) + 3;  // + accf, rready, rfull
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
-    static constexpr int SF_COLS_STAGE = 2 * SF_ATOMS * 4;  // A then B scale tiles, 4 columns each
+    static constexpr int SLOT_COLS = 2 * SF_ATOMS * 4;  // per B stage: A then B scale tiles
     static constexpr int SF_TMEM_BASE = BN;
     static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr int STG_BYTES = 32 * 64;           // per epilogue warp: 32 rows x 32 bf16 columns
     static_assert(KSTEPS == 4, "4 MMAs per stage");
-    static_assert(SF_TMEM_BASE + STAGES * SF_COLS_STAGE <= static_cast<int>(TMEM_COLS), "TMEM budget");
-    static_assert((kMaxSplits - 1) * 128 * BN * 4 <= OFF_TAB, "reduction buffer inside the ring");
+    static_assert(XSLOTS % XPS == 0, "whole stages in the bf16 ring");
+    static_assert(SF_TMEM_BASE + BSTAGES * SLOT_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
+    static_assert((kMaxSplits - 1) * 128 * BN * 4 <= OFF_TAB, "reduction buffer inside the rings");
+    static_assert(QWARPS * STG_BYTES <= OFF_TAB, "output staging inside the rings");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int KIND, bool OUT_F32, int QRULE>
 __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     gemm_rowq_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_b,
-                     const GemmArgs p) {
+                     const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
     using C = RowqCfg<KIND>;
-    constexpr int STAGES = C::STAGES, BN = C::BN;
+    constexpr int BN = C::BN, XS = C::XSLOTS, AS = C::ASTAGES, BSt = C::BSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* qready = full + STAGES;
-    uint64_t* empty = qready + STAGES;
-    uint64_t* accf = empty + STAGES;
-    uint64_t* rready = accf + 1;  // non-leaders: the leader's ring is free for the partials
+    uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* xempty = xfull + XS;
+    uint64_t* aready = xempty + XS;
+    uint64_t* aempty = aready + AS;
+    uint64_t* bfull = aempty + AS;
+    uint64_t* bempty = bfull + BSt;
+    uint64_t* accf = bempty + BSt;
+    uint64_t* rready = accf + 1;  // non-leaders: the leader's rings are free for the partials
     uint64_t* rfull = accf + 2;   // leader: every partial has landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
     float* tab_d = reinterpret_cast<float*>(smem + C::OFF_TAB);
@@ -1199,10 +1227,17 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tma_x);
         prefetch_tmap(&tma_b);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&qready[s], C::QWARPS);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], C::QWARPS);
+        }
+        for (int s = 0; s < AS; ++s) {
+            mbar_init(&aready[s], C::QWARPS);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int s = 0; s < BSt; ++s) {
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bempty[s], 1);
         }
         mbar_init(accf, 1);
         mbar_init(rready, 1);
@@ -1223,47 +1258,66 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     if (warp == 0) {
-        // TMA producer: the whole warp runs the loop; one elected lane issues
-        const uint64_t pol_x = policy_evict_first();
-        const uint64_t pol_b = policy_evict_last();
+        // bf16 producer: slot (stage - k0) * XPS + b, b the 64-element box of the stage
+        const uint64_t pol = policy_evict_first();
+        int slot = 0;
+        uint32_t phase = 0;
+        for (int ks = k0; ks < k1; ++ks) {
+            for (int b = 0; b < C::XPS; ++b) {
+                if (!mbar_wait_warp(&xempty[slot], phase ^ 1u, p.status, 41)) {
+                    ks = k1;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&xfull[slot], C::X_BYTES);
+                    tma_load_2d(&tma_x, &xfull[slot], smem + C::OFF_X + slot * C::X_BYTES, (ks * C::BK + b * 64) * 2,
+                                mt * 128, pol);
+                }
+                __syncwarp();
+                if (++slot == XS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // weight producer
+        const uint64_t pol = policy_evict_last();
         int stage = 0;
         uint32_t phase = 0;
         for (int ks = k0; ks < k1; ++ks) {
-            if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status, 41)) break;
+            if (!mbar_wait_warp(&bempty[stage], phase ^ 1u, p.status, 48)) break;
             if (elect_one()) {
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
-                mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::B_BYTES + atoms * 512);
-#pragma unroll
-                for (int b = 0; b < C::X_BOXES; ++b)
-                    tma_load_2d(&tma_x, &full[stage], smem + C::OFF_X + stage * C::X_BYTES + b * 128 * 128,
-                                (ks * C::BK + b * 64) * 2, mt * 128, pol_x);
-                tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, 0, pol_b);
+                mbar_arrive_expect_tx(&bfull[stage], C::B_BYTES + atoms * 512);
+                tma_load_2d(&tma_b, &bfull[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, 0, pol);
                 bulk_load(smem + C::OFF_SFB + stage * C::SF_BYTES,
-                          p.b_sf + static_cast<int64_t>(ks) * C::SF_ATOMS * 512, atoms * 512, &full[stage]);
+                          p.b_sf + static_cast<int64_t>(ks) * C::SF_ATOMS * 512, atoms * 512, &bfull[stage]);
             }
             __syncwarp();
-            if (++stage == STAGES) {
+            if (++stage == BSt) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
     } else if (warp == 1) {
         // scale copies and MMAs: the whole warp runs the loop; one elected lane issues
-        int stage = 0;
-        uint32_t phase = 0;
+        int as = 0, bs = 0;
+        uint32_t aph = 0, bph = 0;
         bool ok = true;
         for (int ks = k0; ks < k1; ++ks) {
-            if (!mbar_wait_warp(&full[stage], phase, p.status, 42) ||
-                !mbar_wait_warp(&qready[stage], phase, p.status, 43)) {
+            if (!mbar_wait_warp(&bfull[bs], bph, p.status, 42) || !mbar_wait_warp(&aready[as], aph, p.status, 43)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
-            const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SF_BYTES);
-            const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SF_BYTES);
-            const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-            const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+            // TMEM scale slot of this B stage (free: its previous MMAs completed before the
+            // producer could refill the stage)
+            const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + bs * C::SLOT_COLS;
+            const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + as * C::SF_BYTES);
+            const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + bs * C::SF_BYTES);
+            const uint32_t a_s = smem_u32(smem + C::OFF_A + as * C::A_BYTES);
+            const uint32_t b_s = smem_u32(smem + C::OFF_B + bs * C::B_BYTES);
             if (elect_one()) {
 #pragma unroll
                 for (int a = 0; a < C::SF_ATOMS; ++a) {
@@ -1282,12 +1336,17 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
                                                (ks > k0 || j > 0) ? 1u : 0u);
                     }
                 }
-                tc_commit(&empty[stage]);
+                tc_commit(&aempty[as]);
+                tc_commit(&bempty[bs]);
             }
             __syncwarp();
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
+            if (++as == AS) {
+                as = 0;
+                aph ^= 1u;
+            }
+            if (++bs == BSt) {
+                bs = 0;
+                bph ^= 1u;
             }
         }
         if (ok && elect_one()) tc_commit(accf);
@@ -1295,10 +1354,10 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     } else {
         // quantizers: thread qt takes units (row, j) of 32 elements, a warp 32 consecutive rows of
         // one unit column, so its 16-byte reads of the swizzled bf16 rows fall in distinct banks
-        static_assert(128 * (C::BK / 32) % (32 * C::QWARPS) == 0, "whole units per thread");
-        const int qt = (warp - 2) * 32 + lane;
-        constexpr int UPR = C::BK / 32;                 // units per row and stage
+        const int qt = (warp - 3) * 32 + lane;
+        constexpr int UPR = C::BK / 32;                    // units per row and stage
         constexpr int UPT = 128 * UPR / (32 * C::QWARPS);  // units per thread and stage
+        static_assert(128 * UPR % (32 * C::QWARPS) == 0, "whole units per thread");
         float g_a = 1.0f;
         if constexpr (KIND == 1) {
             g_a = *p.g_a;
@@ -1309,20 +1368,26 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
             }
             named_barrier_sync(1, 32 * C::QWARPS);
         }
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int ks = k0; ks < k1; ++ks) {
-            if (!mbar_wait_warp(&full[stage], phase, p.status, 44)) break;
-            const uint32_t x_s = smem_u32(smem + C::OFF_X + stage * C::X_BYTES);
-            const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-            uint8_t* sfa = smem + C::OFF_SFA + stage * C::SF_BYTES;
+        int xslot = 0, as = 0;
+        uint32_t xph = 0, aph = 0;
+        bool ok = true;
+        for (int ks = k0; ks < k1 && ok; ++ks) {
+#pragma unroll
+            for (int b = 0; b < C::XPS; ++b) {
+                const int sl = (xslot + b) % XS;
+                const uint32_t ph = xph ^ static_cast<uint32_t>((xslot + b) / XS);
+                ok = ok && mbar_wait_warp(&xfull[sl], ph & 1u, p.status, 44);
+            }
+            if (!ok || !mbar_wait_warp(&aempty[as], aph ^ 1u, p.status, 49)) break;
+            const uint32_t a_s = smem_u32(smem + C::OFF_A + as * C::A_BYTES);
+            uint8_t* sfa = smem + C::OFF_SFA + as * C::SF_BYTES;
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const int v = qt + u * 32 * C::QWARPS;
                 const int row = v & 127, j = v >> 7;
                 if (static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
                 uint32_t w[16];
-                const uint32_t rb = x_s + (j >> 1) * 128 * 128 + row * 128;
+                const uint32_t rb = smem_u32(smem + C::OFF_X + ((xslot + (j >> 1)) % XS) * C::X_BYTES) + row * 128;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint4 t = ld_shared_v4(rb + ((((j & 1) * 4 + i) ^ (row & 7)) << 4));
@@ -1351,28 +1416,39 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
             }
             fence_proxy_async_smem();  // the A tile and scale tiles are read next by the tensor core
             __syncwarp();
-            if (lane == 0) mbar_arrive(&qready[stage]);
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
+            if (lane == 0) {
+                mbar_arrive(&aready[as]);
+#pragma unroll
+                for (int b = 0; b < C::XPS; ++b) mbar_arrive(&xempty[(xslot + b) % XS]);
+            }
+            xslot += C::XPS;
+            if (xslot >= XS) {
+                xslot -= XS;
+                xph ^= 1u;
+            }
+            if (++as == AS) {
+                as = 0;
+                aph ^= 1u;
             }
         }
     }
 
-    // reduction and epilogue: warps 2-17 hold 32 accumulator columns of one TMEM sub-partition each;
-    // the leader frees its ring for the partials once its MMAs are done, the others send their
-    // valid rows with st.async (column-quad-major layout, as in the split-K kernel) and leave
+    // reduction and epilogue: warps 3-18 hold 32 accumulator columns of one TMEM sub-partition
+    // each; the leader frees its rings for the partials once its MMAs are done, the others send
+    // their valid rows with st.async (column-quad-major layout, as in the split-K kernel) and
+    // leave; the leader adds them in split order and stores through a staging tile per warp and a
+    // TMA store (rows per lane, so direct stores would touch one sector per element)
     constexpr int COLS = BN / (C::QWARPS / 4);
-    const bool epi = warp >= 2;
+    const bool epi = warp >= 3;
     const int sub = warp & 3;
-    const int col0 = ((warp - 2) >> 2) * COLS;
+    const int col0 = ((warp - 3) >> 2) * COLS;
     const int row = sub * 32 + lane;
     float* red = reinterpret_cast<float*>(smem);
     float acc[COLS];
     cluster_wait();  // every CTA of the cluster has initialised its barriers
     if (epi) {
         const bool ok = mbar_wait(accf, 0, p.status, 45);
-        if (split == 0 && warp == 2 && lane == 0)
+        if (split == 0 && warp == 3 && lane == 0)
             for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
         tc_fence_after();
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
@@ -1393,9 +1469,9 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
         for (int v = 0; v < COLS / 4; ++v)
             st_async_v4(dst + v * 128 * 16, acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3], bar);
     }
-    if (epi && split == 0 && row < mrows) {
-        const bool got = mbar_wait(rfull, 0, p.status, 47);
-        for (uint32_t sp = 1; got && sp < splits; ++sp) {
+    if (epi && split == 0) {
+        const bool got = row < mrows ? mbar_wait(rfull, 0, p.status, 47) : true;
+        for (uint32_t sp = 1; got && row < mrows && sp < splits; ++sp) {
             const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (BN / 4) + col0 / 4) * 128 + row;
 #pragma unroll
             for (int v = 0; v < COLS / 4; ++v) {
@@ -1409,18 +1485,42 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
         const int64_t m = static_cast<int64_t>(mt) * 128 + row;
         if constexpr (!OUT_F32) {
-            uint16_t* o16 = reinterpret_cast<uint16_t*>(p.out) + m * p.N;
+            uint32_t packed[COLS / 2];
 #pragma unroll
             for (int i = 0; i < COLS / 2; ++i) {
                 const float lo = KIND == 1 ? __fmul_rn(acc[2 * i], alpha) : acc[2 * i];
                 const float hi = KIND == 1 ? __fmul_rn(acc[2 * i + 1], alpha) : acc[2 * i + 1];
                 const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-                const uint32_t pk = *reinterpret_cast<const uint32_t*>(&b);
-                const int n = col0 + 2 * i;
-                if (n < p.N) o16[n] = static_cast<uint16_t>(pk & 0xFFFFu);
-                if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(pk >> 16);
+                packed[i] = *reinterpret_cast<const uint32_t*>(&b);
             }
-        } else {
+            if (p.tma_store) {
+                // every epilogue warp is done reading the partials before the staging tiles reuse them
+                named_barrier_sync(2, 32 * C::QWARPS);
+                // 32 rows x 32 columns per warp, 64B swizzle (16-byte piece q of row r at q ^ ((r >> 1) & 3))
+                uint8_t* stg = smem + (warp - 3) * C::STG_BYTES;
+                const uint32_t st_row = smem_u32(stg) + lane * 64;
+                const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(st_row + ((q ^ sw) << 4),
+                                 make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && sub * 32 < mrows && col0 < p.N) {
+                    tma_store_2d(&tma_out, stg, col0, mt * 128 + sub * 32);  // clipped at the M and N edges
+                    bulk_commit_group();
+                    bulk_wait_group0();
+                }
+            } else if (row < mrows) {
+                uint16_t* o16 = reinterpret_cast<uint16_t*>(p.out) + m * p.N;
+#pragma unroll
+                for (int i = 0; i < COLS / 2; ++i) {
+                    const int n = col0 + 2 * i;
+                    if (n < p.N) o16[n] = static_cast<uint16_t>(packed[i] & 0xFFFFu);
+                    if (n + 1 < p.N) o16[n + 1] = static_cast<uint16_t>(packed[i] >> 16);
+                }
+            }
+        } else if (row < mrows) {
             float* orow = static_cast<float*>(p.out) + m * p.N;
 #pragma unroll
             for (int i = 0; i < COLS; ++i)
@@ -1984,15 +2084,35 @@ int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cuda
     return MXQ_OK;
 }
 
+// bf16 out [M][N] in boxes of 128 columns x 32 rows, no swizzle (the few-token kernel's output
+// tile); TMA stores clip at the M and N edges.  Needs N % 8 == 0.
+bool make_out_tok_map(CUtensorMap* m, void* base, int64_t M, int64_t N) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {128, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <int KIND, bool F32, int QRULE>
 int run_decode(const void* x, const void* B_q, GemmArgs args, int splits, cudaStream_t stream) {
     using C = DecCfg<KIND>;
     auto kern = gemm_decode_kernel<KIND, F32, QRULE>;
-    CUtensorMap tx, tw;
+    CUtensorMap tx, tw, to;
     // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 32 rows; W codes 128 rows x 128 bytes
     if (!make_map(&tx, x, 2 * static_cast<uint64_t>(args.K), args.M, C::TOK) ||
         !make_map(&tw, B_q, args.K / C::EPB, args.N, 128))
         return MXQ_ERR_CUDA;
+    memset(&to, 0, sizeof(to));
+    args.tma_store = 0;
+    if (!F32 && args.N % 8 == 0) {
+        if (!make_out_tok_map(&to, args.out, args.M, args.N)) return MXQ_ERR_CUDA;
+        args.tma_store = 1;
+    }
     args.m_tiles = 1;
     args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
@@ -2019,19 +2139,39 @@ int run_decode(const void* x, const void* B_q, GemmArgs args, int splits, cudaSt
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tx, tw, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tw, to, args) != cudaSuccess) return MXQ_ERR_CUDA;
     return MXQ_OK;
+}
+
+// bf16 out [M][N] in boxes of 32 columns (64 bytes) x 32 rows, 64B swizzle (16-byte piece q of row
+// r at piece q ^ ((r >> 1) & 3)); TMA stores clip at the M and N edges.  Needs N % 8 == 0.
+bool make_out32_map(CUtensorMap* m, void* base, int64_t M, int64_t N) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
 }
 
 template <int KIND, bool F32, int QRULE>
 int run_rowq(const void* x, const void* B_q, GemmArgs args, int splits, cudaStream_t stream) {
     using C = RowqCfg<KIND>;
     auto kern = gemm_rowq_kernel<KIND, F32, QRULE>;
-    CUtensorMap tx, tb;
+    CUtensorMap tx, tb, to;
     // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 128 rows; W codes as the GEMM's
     if (!make_map(&tx, x, 2 * static_cast<uint64_t>(args.K), args.M, 128) ||
         !make_map(&tb, B_q, args.K / C::EPB, args.N, 128))
         return MXQ_ERR_CUDA;
+    memset(&to, 0, sizeof(to));
+    args.tma_store = 0;
+    if (!F32 && args.N % 8 == 0) {
+        if (!make_out32_map(&to, args.out, args.M, args.N)) return MXQ_ERR_CUDA;
+        args.tma_store = 1;
+    }
     args.m_tiles = static_cast<int>(ceil_div(args.M, 128));
     args.n_tiles = 1;
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
@@ -2058,7 +2198,7 @@ int run_rowq(const void* x, const void* B_q, GemmArgs args, int splits, cudaStre
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tx, tb, args) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tb, to, args) != cudaSuccess) return MXQ_ERR_CUDA;
     return MXQ_OK;
 }
 
