@@ -802,9 +802,8 @@ struct DecCfg {
     static constexpr int KB_PER_MMA = MMA_K / BS;
     static constexpr int SF_ATOMS = BK / BS / 4;
     static constexpr int TOK = 32;                   // MMA N: token rows (rows >= M are zero)
-    // a deep weight ring: about 112 KB per SM in flight is what the HBM latency under this load
-    // needs (with 5 stages the first stage of every CTA arrived only after about 2.3 us)
-    static constexpr int WSTAGES = (KIND == 1) ? 6 : 7, XSTAGES = 2, TSTAGES = 5;
+    // 4 to 7 weight stages measured the same (graph replays with the weights streamed from HBM)
+    static constexpr int WSTAGES = 5, XSTAGES = 2, TSTAGES = 5;
     static constexpr int W_BYTES = 128 * 128;
     static constexpr int SF_BYTES = SF_ATOMS * 512;
     static constexpr int X_BOXES = BK / 64;
