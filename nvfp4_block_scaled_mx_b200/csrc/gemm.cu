@@ -3,9 +3,11 @@
 // Three kernels share the MMA, scale and epilogue plumbing, chosen on the host by shape:
 //   gemm_pair_kernel    M > 128: two-CTA clusters computing 256 x BN tiles (cta_group::2);
 //   gemm_splitk_kernel  M <= 128 with too few output tiles for the SMs: K split over a cluster,
-//                       partials reduced through distributed shared memory (and, for up to 32
-//                       rows, the activations quantized inside the kernel);
+//                       partials reduced through distributed shared memory;
 //   gemm_kernel         M <= 128 otherwise, described here.
+// Two more kernels serve the linear layer in one launch, quantizing its bf16 activations themselves:
+//   gemm_decode_kernel  up to 32 tokens (weights as the 128-row MMA operand, tokens as N = 32);
+//   gemm_rowq_kernel    more tokens and N <= 128 (each activation row read once, as bf16).
 //
 // gemm_kernel: one persistent CTA per SM, warp-specialised:
 //   warp 0       TMA producer: A and B tiles (128-byte K slices, 128B-swizzled) and their
@@ -102,8 +104,7 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
     static constexpr int N_BARS = 3 * STAGES + 2 * ACC_STAGES;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
-    static constexpr int OFF_TAB = OFF_SLOT + 16;             // NVFP4 d and 1/d tables (in-kernel quantizer)
-    static constexpr int SMEM_BYTES = OFF_TAB + 1024 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;  // + slack for 1024-byte alignment
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -447,16 +448,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr uint32_t kMaxSplits = 4;
 
-// QRULE >= 0 (M <= 32): A is not pre-quantized.  TMA brings the stage's bf16 activations (boxes of
-// 64 elements x rows, 128B swizzle; at most 32 rows x BK x 2 bytes = the stage's A buffer) and the
-// scale-staging warps quantize them in place into the A tile and the A scale tiles (rule QRULE for
-// MX formats) with the streaming quantizer's arithmetic, so a few-token linear layer is one launch.
-template <int KIND, bool OUT_F32, int QRULE = -1>
+template <int KIND, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                        const GemmArgs p) {
     constexpr int BN = 128, STAGES = 6;
-    constexpr bool QA = QRULE >= 0;
     using C = Cfg<KIND, BN, STAGES>;
     static_assert((kMaxSplits - 1) * 128 * BN * 4 <= STAGES * (C::A_BYTES + C::B_BYTES), "reduction buffer");
     extern __shared__ uint8_t smem_raw[];
@@ -514,17 +510,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (elect_one()) {
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
                 // A rows past M are not loaded: they only feed accumulator rows that are never stored
-                constexpr int A_BOXES = QA ? C::BK / 64 : 1;  // bf16 boxes of 64 elements, or one FP4/FP8 box
-                mbar_arrive_expect_tx(&full[stage], A_BOXES * p.a_box_bytes + C::B_BYTES +
-                                                        atoms * 512 * ((QA ? 0 : 1) + (b_group ? 1 : 0)));
-#pragma unroll
-                for (int b = 0; b < A_BOXES; ++b)
-                    tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES + b * p.a_box_bytes,
-                                (QA ? ks * C::BK * 2 : ks * 128) + b * 128, 0, pol);
+                mbar_arrive_expect_tx(&full[stage], p.a_box_bytes + C::B_BYTES + atoms * 512 * (1 + (b_group ? 1 : 0)));
+                tma_load_2d(&tma_a, &full[stage], smem + C::OFF_A + stage * C::A_BYTES, ks * 128, 0, pol);
                 tma_load_2d(&tma_b, &full[stage], smem + C::OFF_B + stage * C::B_BYTES, ks * 128, nt * BN, pol);
                 const int64_t kcol = static_cast<int64_t>(ks) * C::SF_ATOMS;
-                if (!QA)
-                    bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, p.a_sf + kcol * 512, atoms * 512, &full[stage]);
+                bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, p.a_sf + kcol * 512, atoms * 512, &full[stage]);
                 if (b_group)
                     bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES,
                               p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + kcol) * 512, atoms * 512,
@@ -573,92 +563,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && elect_one()) tc_commit(accf);
         __syncwarp();
-    } else if (warp >= 2 + kEpiWarps || (QA && warp >= 6 && warp < 2 + kEpiWarps)) {
-        // scale staging (warps 10-13, one per TMEM sub-partition).  With the in-kernel quantizer
-        // epilogue warps 6-9 (again one per sub-partition) form a second group, and the two groups
-        // take alternate stages, so that one group's barrier and load latencies sit under the other's
+    } else if (warp >= 2 + kEpiWarps) {
+        // scale staging (warps 10-13, one per TMEM sub-partition)
         const int sub = warp & 3;
         const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
-        const int grp = warp >= 2 + kEpiWarps ? 0 : 1;
-        const int bar_id = 1 + grp;
         int stage = 0;
         uint32_t phase = 0;
-        // in-kernel quantizer: thread qt of the group's 4 warps takes units (row, j) of 32 elements
-        const int qt = (warp & 3) * 32 + lane;
-        constexpr int UPR = C::BK / 32;  // 32-element units per row and stage
-        constexpr int UPT = 32 * UPR / 128;  // units per thread at most (M <= 32)
-        float* tab_d = reinterpret_cast<float*>(smem + C::OFF_TAB);
-        float* tab_r = tab_d + 128;
-        float g_a = 1.0f;
-        if constexpr (QA && KIND == 1) {
-            g_a = *p.g_a;
-            const float d = __fmul_rn(e4m3_decode_pos(static_cast<uint32_t>(qt)), g_a);
-            tab_d[qt] = d;
-            tab_r[qt] = __frcp_rn(d);  // fl(1/d), +inf for d = 0; both groups write the same values
-            named_barrier_sync(bar_id, 4 * 32);
-        }
         for (int ks = k0; ks < k1; ++ks) {
-            if (QA && ((ks - k0) & 1) != grp) {
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-                continue;
-            }
-            if constexpr (QA) {
-                if (named_barrier_or(bar_id, 4 * 32, !mbar_wait(&full[stage], phase, p.status, 26))) break;
-                const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-                uint8_t* sfa = smem + C::OFF_SFA + stage * C::SFA_BYTES;
-                // read this thread's units of bf16 (unit (row, j) = 64 bytes of box j / 2) ...
-                uint32_t w[UPT][16];
-#pragma unroll
-                for (int u = 0; u < UPT; ++u) {
-                    // a warp takes 32 rows of one unit column (conflict-free reads); up to 8 rows, a
-                    // warp takes 4 rows x 8 unit columns (fewer units per thread)
-                    const int v = qt + u * 128;
-                    const int row = p.M > 8 ? (v & 31) : v / UPR, jj = p.M > 8 ? (v >> 5) : v % UPR;
-                    if (row < p.M && static_cast<int64_t>(ks) * C::BK + jj * 32 < p.K) {
-                        const uint32_t rb = a_s + (jj >> 1) * p.a_box_bytes + row * 128;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint4 t = ld_shared_v4(rb + ((((jj & 1) * 4 + i) ^ (row & 7)) << 4));
-                            w[u][4 * i] = t.x;
-                            w[u][4 * i + 1] = t.y;
-                            w[u][4 * i + 2] = t.z;
-                            w[u][4 * i + 3] = t.w;
-                        }
-                    }
-                }
-                named_barrier_sync(bar_id, 4 * 32);  // ... before any thread overwrites the buffer with codes
-#pragma unroll
-                for (int u = 0; u < UPT; ++u) {
-                    const int v = qt + u * 128;
-                    const int row = p.M > 8 ? (v & 31) : v / UPR, j = p.M > 8 ? (v >> 5) : v % UPR;
-                    if (row >= p.M || static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
-                    uint32_t codes[8], seen = 0;
-                    const uint32_t sc =
-                        quantize32<KIND, (QRULE < 0 ? 0 : QRULE), false>(w[u], g_a, tab_d, tab_r, codes, seen);
-                    const uint32_t sw = static_cast<uint32_t>(row & 7);
-                    const uint32_t sf_row = (row & 31) * 16 + ((row >> 5) & 3) * 4;
-                    const uint32_t a_row = a_s + row * 128;
-                    if constexpr (KIND == 2) {  // MXFP8: 32 bytes of codes, one scale block
-                        st_shared_v4(a_row + (((2 * j) ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
-                        st_shared_v4(a_row + (((2 * j + 1) ^ sw) << 4), make_uint4(codes[4], codes[5], codes[6], codes[7]));
-                        sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
-                    } else if constexpr (KIND == 1) {  // NVFP4: 16 bytes of codes, scale blocks 2j and 2j + 1
-                        st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
-                        *reinterpret_cast<uint16_t*>(sfa + ((2 * j) >> 2) * 512 + sf_row + ((2 * j) & 3)) =
-                            static_cast<uint16_t>(sc);
-                    } else {  // MXFP4: 16 bytes of codes, one scale block
-                        st_shared_v4(a_row + ((j ^ sw) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
-                        sfa[(j >> 2) * 512 + sf_row + (j & 3)] = static_cast<uint8_t>(sc);
-                    }
-                }
-                fence_proxy_async_smem();            // the A tile is read next by the tensor cores
-                named_barrier_sync(bar_id, 4 * 32);  // every scale byte of the stage is in shared memory
-            } else if (!mbar_wait(&full[stage], phase, p.status, 26)) {
-                break;
-            }
+            if (!mbar_wait(&full[stage], phase, p.status, 26)) break;
             uint32_t r[C::SF_COLS_STAGE];
 
             const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES) + lane * 16;
@@ -2040,17 +1952,14 @@ int run_pair(const void* A_q, const void* B_q, GemmArgs args, cudaStream_t strea
     return MXQ_OK;
 }
 
-template <int KIND, bool F32, int QRULE = -1>
+template <int KIND, bool F32>
 int run_splitk(const void* A_q, const void* B_q, GemmArgs args, int splits, cudaStream_t stream, bool pdl) {
     using C = Cfg<KIND, 128, 6>;
-    auto kern = gemm_splitk_kernel<KIND, F32, QRULE>;
+    auto kern = gemm_splitk_kernel<KIND, F32>;
     const int row_bytes = args.K / C::EPB;
     CUtensorMap ta, tb;
     const uint32_t a_rows = static_cast<uint32_t>(ceil_div(args.M, 8) * 8);
-    // A is either quantized (row_bytes per row) or, quantized in the kernel, bf16 (2 K bytes per row)
-    if (!make_map(&tb, B_q, row_bytes, args.N, 128) ||
-        !make_map(&ta, QRULE >= 0 ? args.x : A_q, QRULE >= 0 ? 2 * static_cast<uint64_t>(args.K) : row_bytes, args.M,
-                  a_rows))
+    if (!make_map(&tb, B_q, row_bytes, args.N, 128) || !make_map(&ta, A_q, row_bytes, args.M, a_rows))
         return MXQ_ERR_CUDA;
     args.a_box_bytes = a_rows * 128;
     args.m_tiles = 1;
