@@ -9,7 +9,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("M,N,K,fmt", [(300, 512, 1024, "mxfp4"), (32, 1024, 2048, "mxfp4"), (256, 384, 512, "nvfp4"),
-                                       (200, 256, 512, "mxfp8")])
+                                       (200, 256, 512, "mxfp8"), (200, 96, 1024, "mxfp8"), (300, 128, 512, "nvfp4"),
+                                       (8, 2048, 1024, "nvfp4")])
 def test_linear_graph_replay_matches_eager(M, N, K, fmt):
     A1 = synth.random_bf16((M, K), 7).cuda()
     A2 = synth.random_bf16((M, K), 8, std=3.0).cuda()
