@@ -1153,7 +1153,9 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
         mbar_init(accf, 1);
         mbar_init(rready, 1);
         mbar_init(rfull, 1);
-        if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * static_cast<uint32_t>(mrows) * BN * 4);
+        // the partials of the other CTAs: valid rows, and only the 32-column groups below N
+        const uint32_t groups = static_cast<uint32_t>(min(BN, (p.N + 31) & ~31) / 32);
+        if (split == 0) mbar_arrive_expect_tx(rfull, (splits - 1) * static_cast<uint32_t>(mrows) * groups * 32 * 4);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1373,7 +1375,8 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
         }
         tc_fence_before();
     }
-    if (epi && split != 0 && row < mrows && mbar_wait_cluster(rready, 0, p.status, 46)) {
+    static_assert(COLS == 32, "one 32-column group per epilogue warp");
+    if (epi && split != 0 && row < mrows && col0 < p.N && mbar_wait_cluster(rready, 0, p.status, 46)) {
         const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (BN / 4) + col0 / 4) * 128 + row) * 4), 0);
         const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
 #pragma unroll
@@ -1382,7 +1385,7 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     }
     if (epi && split == 0) {
         const bool got = row < mrows ? mbar_wait(rfull, 0, p.status, 47) : true;
-        for (uint32_t sp = 1; got && row < mrows && sp < splits; ++sp) {
+        for (uint32_t sp = 1; got && row < mrows && col0 < p.N && sp < splits; ++sp) {
             const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (BN / 4) + col0 / 4) * 128 + row;
 #pragma unroll
             for (int v = 0; v < COLS / 4; ++v) {

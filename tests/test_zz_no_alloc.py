@@ -30,17 +30,20 @@ def _noalloc(x, Wq, Wsf, N, fmt, rule, out, g_w=None, g_a=None):
                                         mxq.RULE[rule], ot, p(out), torch.cuda.current_stream().cuda_stream)
 
 
+# N = 384 with 200 and 37 tokens takes the quantizer + GEMM path (the array holds the quantized
+# activations); N = 96 and 17 tokens take the one-launch kernels that quantize inside the GEMM
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_noalloc_matches_linear_two_calls(fmt, out_dtype):
-    N, K = 384, 1024
+@pytest.mark.parametrize("N,calls", [(384, ((200, 11), (37, 12))), (96, ((200, 13), (17, 14)))])
+def test_noalloc_matches_linear_two_calls(fmt, out_dtype, N, calls):
+    K = 1024
     W = synth.random_bf16((N, K), 5, std=0.02).cuda()
     g_w = None
     if fmt == "nvfp4":
         g_w, _ = mxq.global_scale(W)
     Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w, layout=mxq.SF_SWIZZLED)
     Wq_ref, Wsf_ref = oracle_quantize(W.cpu(), fmt, "even", float(g_w.item()) if g_w is not None else 1.0)
-    for M, seed in [(200, 11), (37, 12)]:
+    for M, seed in calls:
         A = synth.random_bf16((M, K), seed).cuda()
         g_a = None
         if fmt == "nvfp4":
