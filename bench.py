@@ -76,6 +76,15 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def sustained_bf16_tflops():
+    """The measured bf16 GEMM rate in a seconds-long loop under the power cap (None if unknown)."""
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as fh:
+            v = json.load(fh).get("bf16_tflops_sustained")
+        return float(v) if v else None
+    return None
+
+
 def traffic_for(key):
     if os.path.exists(TRAFFIC_PATH):
         with open(TRAFFIC_PATH) as fh:
@@ -158,14 +167,19 @@ class ClockSampler:
         rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        num = lambda v: float(v) if v.strip().replace(".", "").isdigit() else None
+        smp = [(num(r[1]), num(r[3])) for r in rows]
+        smp = [(c, w) for c, w in smp if c is not None and w is not None]
         smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
-        # the timed region is the busy part of the sampling window: report the upper half
-        busy = sorted(sm)[len(sm) // 2:] if sm else []
-        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+        # the samples under load (power draw at least half the window's maximum); the idle moments
+        # before and after the timed region run at the top clock and would hide a power-capped clock
+        top = max((w for _, w in smp), default=0.0)
+        load = [c for c, w in smp if w >= 0.5 * top]
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": top if smp else None}
 
 
 # ---------------------------------------------------------------- the mxq arm
@@ -314,6 +328,9 @@ def run_mxq(args, world, rank, local):
                 "peak_source": "%s bf16 %.1f TFLOP/s x %g nominal %s:bf16 ratio" % (
                     peak_src, bf16_tflops, FP4_PER_BF16 if fmt != "mxfp8" else FP8_PER_BF16, fmt),
                 "frac_of_datasheet": round(gemm_tflops / (9000.0 if fmt != "mxfp8" else 4500.0), 4),
+                "frac_of_sustained_peak": (round(gemm_tflops / (sustained_bf16_tflops() * (FP8_PER_BF16 if fmt == "mxfp8"
+                                                                                           else FP4_PER_BF16)), 4)
+                                           if sustained_bf16_tflops() else None),
                 "traffic": traffic_for("gemm_%s_%s" % (fmt, workload)),
                 "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
     one_launch = mxq.linear_kernel_count(M, N, K, fmt) == 1

@@ -76,3 +76,20 @@ def test_reference_arm_prints_the_contract_line():
     assert d["config"]["workload"] == "prefill_gate_up"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_summary_uses_the_samples_under_load():
+    """The bench reports the median SM clock of the samples taken under load (power at least half the
+    window's maximum): the idle moments around the timed region run at the top clock and must not
+    hide a power-capped clock; throttle reasons seen anywhere in the window are reported."""
+    import bench
+    c = bench.ClockSampler(0)
+    c.out = ("0, 1965, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+             "0, 1500, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+             "0, 1450, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+             "0, 1965, 1965, 130.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    s = c.summary()
+    assert s["sm_mhz"] == 1475.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples_under_load"] == 2
+    c.out = ""
+    assert c.summary()["reasons"] == ["unsampled"]
