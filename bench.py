@@ -344,7 +344,7 @@ def run_mxq(args, world, rank, local):
                                                        g_W=g_w, g_A=g_a, workspace=ws, out=out, stream=stream),
                                     20, stream, flush)
             gbytes = W_q.numel() + W_sf.numel() + 2 * M * K + out.numel() * out.element_size()
-            kname = ("gemm_splitk_kernel (tcgen05 kind::%s, few tokens, activations quantized in the kernel)" if M <= 32
+            kname = ("gemm_decode_kernel (tcgen05 kind::%s, few tokens, activations quantized in the kernel)" if M <= 32
                      else "gemm_rowq_kernel (tcgen05 kind::%s, few columns, activations quantized in the kernel)") % kind
         else:
             lin_cold = time_flushed(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a,
@@ -354,7 +354,8 @@ def run_mxq(args, world, rank, local):
         roofline = {"bound": "hbm", "kernel": kname,
                     "achieved": round(gbytes / lin_cold / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
                     "frac": round(gbytes / lin_cold / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
-                    "traffic": None, "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(lin_cold * 1e3, 4),
+                    "traffic": traffic_for("linear_%s_%s" % (fmt, workload)) if one_launch else None,
+                    "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(lin_cold * 1e3, 4),
                     "l2": "flushed per launch (the launch latency is inside the time)"}
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
