@@ -706,7 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warps 3-10   quantize the token stages into the token-code ring (B operand layout) with the
 //                streaming quantizer's arithmetic; then the epilogue.  Partials of the non-leader
 //                CTAs go to a buffer of their own in the leader as soon as they are ready.
-template <int KIND>
+// WG = 2 (many weight rows, no K split): a CTA owns 256 weight rows as two 128-row MMA groups with an
+// accumulator each, so that the tiles fit one wave and the tokens are quantized once per 256 rows.
+template <int KIND, int WG>
 struct DecCfg {
     static constexpr int BS = Fmt<KIND>::BS, EPB = Fmt<KIND>::EPB, MMA_K = Fmt<KIND>::MMA_K;
     static constexpr int BK = 128 * EPB;
@@ -715,41 +717,42 @@ struct DecCfg {
     static constexpr int SF_ATOMS = BK / BS / 4;
     static constexpr int TOK = 32;                   // MMA N: token rows (rows >= M are zero)
     // 4 to 7 weight stages measured the same (graph replays with the weights streamed from HBM)
-    static constexpr int WSTAGES = 5, XSTAGES = 2, TSTAGES = 5;
-    static constexpr int W_BYTES = 128 * 128;
-    static constexpr int SF_BYTES = SF_ATOMS * 512;
+    static constexpr int WSTAGES = (WG == 1) ? 5 : 4, XSTAGES = 2, TSTAGES = 5;
+    static constexpr int W_BYTES = WG * 128 * 128;
+    static constexpr int SF_BYTES = SF_ATOMS * 512;   // one 128-row scale tile column per stage
+    static constexpr int SFW_BYTES = WG * SF_BYTES;   // the weight groups' scale tiles
     static constexpr int X_BOXES = BK / 64;
     static constexpr int X_BYTES = X_BOXES * TOK * 128;
     static constexpr int T_BYTES = TOK * 128;
     static constexpr int QWARPS = 8;
     static constexpr int THREADS = (3 + QWARPS) * 32;
-    static constexpr int RED_BYTES = (kMaxSplits - 1) * 128 * TOK * 4;
+    static constexpr int RED_BYTES = (WG == 1) ? (kMaxSplits - 1) * 128 * TOK * 4 : 0;  // WG = 2: no K split
     static constexpr int OFF_W = 0;
     static constexpr int OFF_X = OFF_W + WSTAGES * W_BYTES;
     static constexpr int OFF_T = OFF_X + XSTAGES * X_BYTES;
     static constexpr int OFF_RED = OFF_T + TSTAGES * T_BYTES;
     static constexpr int OFF_SFW = OFF_RED + RED_BYTES;
-    static constexpr int OFF_SFT = OFF_SFW + WSTAGES * SF_BYTES;
+    static constexpr int OFF_SFT = OFF_SFW + WSTAGES * SFW_BYTES;
     static constexpr int OFF_TAB = OFF_SFT + TSTAGES * SF_BYTES;
     static constexpr int OFF_BAR = OFF_TAB + 1024;
     static constexpr int N_BARS = 2 * (WSTAGES + XSTAGES + TSTAGES) + 2;  // + accf, rfull
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
-    static constexpr int SLOT_COLS = 2 * SF_ATOMS * 4;  // per weight stage: weight then token scale tiles
-    static constexpr int SF_TMEM_BASE = 32;
+    static constexpr int SLOT_COLS = (WG + 1) * SF_ATOMS * 4;  // per weight stage: weight then token scale tiles
+    static constexpr int SF_TMEM_BASE = WG * 32;                // one 32-column accumulator per weight group
     static constexpr uint32_t TMEM_COLS = 256;
     static_assert(KSTEPS == 4, "4 MMAs per stage");
     static_assert(SF_TMEM_BASE + WSTAGES * SLOT_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
     static_assert(OFF_W % 1024 == 0 && OFF_X % 1024 == 0 && OFF_T % 1024 == 0, "swizzled buffers 1024-aligned");
-    static_assert(TOK * 128 * 2 <= XSTAGES * X_BYTES, "output staging tile inside the token ring");
+    static_assert(WG * TOK * 128 * 2 <= XSTAGES * X_BYTES, "output staging tiles inside the token ring");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int KIND, bool OUT_F32, int QRULE>
-__global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
+template <int KIND, int WG, bool OUT_F32, int QRULE>
+__global__ void __launch_bounds__(DecCfg<KIND, WG>::THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_w,
                        const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
-    using C = DecCfg<KIND>;
+    using C = DecCfg<KIND, WG>;
     constexpr int WS = C::WSTAGES, XS = C::XSTAGES, TS = C::TSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -814,11 +817,15 @@ __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
             if (!mbar_wait_warp(&wempty[stage], phase ^ 1u, p.status, 51)) break;
             if (elect_one()) {
                 const int atoms = min(C::SF_ATOMS, p.sf_col_tiles - ks * C::SF_ATOMS);
-                mbar_arrive_expect_tx(&wfull[stage], C::W_BYTES + atoms * 512);
-                tma_load_2d(&tma_w, &wfull[stage], smem + C::OFF_W + stage * C::W_BYTES, ks * 128, nt * 128, pol);
-                bulk_load(smem + C::OFF_SFW + stage * C::SF_BYTES,
-                          p.b_sf + (static_cast<int64_t>(nt) * p.sf_col_tiles + static_cast<int64_t>(ks) * C::SF_ATOMS) * 512,
-                          atoms * 512, &wfull[stage]);
+                // row groups past N (WG = 2, last tile) load nothing: their rows are TMA zero fill
+                const int groups = min(WG, p.b_row_tiles - nt * WG);
+                mbar_arrive_expect_tx(&wfull[stage], C::W_BYTES + groups * atoms * 512);
+                tma_load_2d(&tma_w, &wfull[stage], smem + C::OFF_W + stage * C::W_BYTES, ks * 128, nt * 128 * WG, pol);
+                for (int g = 0; g < groups; ++g)
+                    bulk_load(smem + C::OFF_SFW + stage * C::SFW_BYTES + g * C::SF_BYTES,
+                              p.b_sf + (static_cast<int64_t>(nt * WG + g) * p.sf_col_tiles +
+                                        static_cast<int64_t>(ks) * C::SF_ATOMS) * 512,
+                              atoms * 512, &wfull[stage]);
             }
             __syncwarp();
             if (++stage == WS) {
@@ -839,27 +846,35 @@ __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
             tc_fence_after();
             // TMEM scale slot of this weight stage (free: its previous MMAs completed before the
             // producer could refill the stage)
+            // slot layout: the weight groups' scale tiles [g][atom], then the token scale tiles [atom]
             const uint32_t slot = tmem_base + C::SF_TMEM_BASE + ws * C::SLOT_COLS;
-            const uint32_t sfw_s = smem_u32(smem + C::OFF_SFW + ws * C::SF_BYTES);
+            const uint32_t sfw_s = smem_u32(smem + C::OFF_SFW + ws * C::SFW_BYTES);
             const uint32_t sft_s = smem_u32(smem + C::OFF_SFT + ts * C::SF_BYTES);
             const uint32_t w_s = smem_u32(smem + C::OFF_W + ws * C::W_BYTES);
             const uint32_t t_s = smem_u32(smem + C::OFF_T + ts * C::T_BYTES);
+            constexpr int SFT_COL = WG * C::SF_ATOMS * 4;
             if (elect_one()) {
 #pragma unroll
                 for (int a = 0; a < C::SF_ATOMS; ++a) {
-                    tc_cp_scales(slot + a * 4, smem_desc(sfw_s + a * 512, 0, 128, kLayoutNone));
-                    tc_cp_scales(slot + C::SF_ATOMS * 4 + a * 4, smem_desc(sft_s + a * 512, 0, 128, kLayoutNone));
+#pragma unroll
+                    for (int g = 0; g < WG; ++g)
+                        tc_cp_scales(slot + (g * C::SF_ATOMS + a) * 4,
+                                     smem_desc(sfw_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                    tc_cp_scales(slot + SFT_COL + a * 4, smem_desc(sft_s + a * 512, 0, 128, kLayoutNone));
                 }
 #pragma unroll
                 for (int j = 0; j < C::KSTEPS; ++j) {
                     if (ks * C::BK + j * C::MMA_K < p.K) {
                         const int kb = j * C::KB_PER_MMA;
                         const int atom = kb >> 2;
-                        mma_block_scaled<KIND>(tmem_base, smem_desc(w_s + j * 32, 16, 1024, kLayoutSwizzle128B),
-                                               smem_desc(t_s + j * 32, 16, 1024, kLayoutSwizzle128B),
-                                               mma_idesc<KIND>(128, C::TOK, static_cast<uint32_t>(kb & 3)),
-                                               slot + atom * 4, slot + C::SF_ATOMS * 4 + atom * 4,
-                                               (ks > k0 || j > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int g = 0; g < WG; ++g)
+                            mma_block_scaled<KIND>(tmem_base + static_cast<uint32_t>(g * C::TOK),
+                                                   smem_desc(w_s + g * 128 * 128 + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                                   smem_desc(t_s + j * 32, 16, 1024, kLayoutSwizzle128B),
+                                                   mma_idesc<KIND>(128, C::TOK, static_cast<uint32_t>(kb & 3)),
+                                                   slot + (g * C::SF_ATOMS + atom) * 4, slot + SFT_COL + atom * 4,
+                                                   (ks > k0 || j > 0) ? 1u : 0u);
                     }
                 }
                 tc_commit(&wempty[ws]);
@@ -969,75 +984,96 @@ __global__ void __launch_bounds__(DecCfg<KIND>::THREADS, 1)
     }
 
     // reduction and epilogue: warp w of 3-10 holds the 16 tokens [16 h, +16) (h = (w - 3) / 4) of the
-    // 32 weight rows in its TMEM sub-partition.  The non-leaders send their partials to the leader's
-    // buffer ([split - 1][token quad][128 rows][4] fp32: a warp's 16-byte stores cover 512
-    // contiguous bytes) as soon as their MMAs are done; the leader adds them in split order.
+    // 32 weight rows in its TMEM sub-partition, for each weight group.  With a K split (WG = 1) the
+    // non-leaders send their partials to the leader's buffer ([split - 1][token quad][128 rows][4]
+    // fp32: a warp's 16-byte stores cover 512 contiguous bytes) as soon as their MMAs are done, and
+    // the leader adds them in split order.
     const bool epi = warp >= 3;
     const int sub = warp & 3;
     const int h = (warp - 3) >> 2;
-    const int wrow = sub * 32 + lane;  // weight row within the tile
+    const int wrow = sub * 32 + lane;  // weight row within a 128-row group
     float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
-    float acc[16];
+    float acc[WG][16];
     cluster_wait();  // every CTA of the cluster has initialised its barriers
     if (epi) {
         const bool ok = mbar_wait(accf, 0, p.status, 57);
         tc_fence_after();
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(16 * h), r);
-        tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = ok ? __uint_as_float(r[i]) : 0.0f;
+        for (int g = 0; g < WG; ++g) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(g * C::TOK + 16 * h),
+                               r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[g][i] = ok ? __uint_as_float(r[i]) : 0.0f;
+        }
         tc_fence_before();
     }
-    if (epi && split != 0) {
-        const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow) * 4), 0);
-        const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
+    if constexpr (WG == 1) {
+        if (epi && split != 0) {
+            const uint32_t dst = mapa_shared(smem_u32(red + (((split - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow) * 4), 0);
+            const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            st_async_v4(dst + q * 128 * 16, acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3], bar);
+            for (int q = 0; q < 4; ++q)
+                st_async_v4(dst + q * 128 * 16, acc[0][4 * q], acc[0][4 * q + 1], acc[0][4 * q + 2], acc[0][4 * q + 3],
+                            bar);
+        }
     }
     if (epi && split == 0) {
         const bool got = mbar_wait(rfull, 0, p.status, 58);
-        for (uint32_t sp = 1; got && sp < splits; ++sp) {
-            const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow;
+        if constexpr (WG == 1) {
+            for (uint32_t sp = 1; got && sp < splits; ++sp) {
+                const float4* src = reinterpret_cast<const float4*>(red) + ((sp - 1) * (C::TOK / 4) + 4 * h) * 128 + wrow;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = src[q * 128];
-                acc[4 * q] = __fadd_rn(acc[4 * q], v.x);
-                acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
-                acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
-                acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+                for (int q = 0; q < 4; ++q) {
+                    const float4 v = src[q * 128];
+                    acc[0][4 * q] = __fadd_rn(acc[0][4 * q], v.x);
+                    acc[0][4 * q + 1] = __fadd_rn(acc[0][4 * q + 1], v.y);
+                    acc[0][4 * q + 2] = __fadd_rn(acc[0][4 * q + 2], v.z);
+                    acc[0][4 * q + 3] = __fadd_rn(acc[0][4 * q + 3], v.w);
+                }
             }
         }
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
-        const int n = nt * 128 + wrow;
         if (!OUT_F32 && p.tma_store) {
-            // the [32 tokens][128 columns] bf16 tile through shared memory (the token ring is idle now:
-            // every stage has been quantized) and one TMA store, clipped at the M and N edges; direct
-            // stores would write one 2-byte element per token row and lane
-            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::OFF_X);
+            // each group's [32 tokens][128 columns] bf16 tile through shared memory (the token ring is
+            // idle now: every stage has been quantized) and one TMA store, clipped at the M and N
+            // edges; direct stores would write one 2-byte element per token row and lane
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float v = KIND == 1 ? __fmul_rn(acc[i], alpha) : acc[i];
-                stg[(16 * h + i) * 128 + wrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            for (int g = 0; g < WG; ++g) {
+                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::OFF_X) + g * C::TOK * 128;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float v = KIND == 1 ? __fmul_rn(acc[g][i], alpha) : acc[g][i];
+                    stg[(16 * h + i) * 128 + wrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                }
             }
             fence_proxy_async_smem();
             named_barrier_sync(2, 32 * C::QWARPS);
             if (warp == 3 && lane == 0) {
-                tma_store_2d(&tma_out, stg, nt * 128, 0);
-                bulk_commit_group();
+                for (int g = 0; g < WG; ++g) {
+                    if ((nt * WG + g) * 128 >= p.N) break;
+                    tma_store_2d(&tma_out, reinterpret_cast<uint16_t*>(smem + C::OFF_X) + g * C::TOK * 128,
+                                 (nt * WG + g) * 128, 0);
+                    bulk_commit_group();
+                }
                 bulk_wait_group0();
             }
-        } else if (n < p.N) {
+        } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int m = 16 * h + i;
-                if (m < p.M) {
-                    const float v = KIND == 1 ? __fmul_rn(acc[i], alpha) : acc[i];
-                    if constexpr (OUT_F32) {
-                        static_cast<float*>(p.out)[static_cast<int64_t>(m) * p.N + n] = v;
-                    } else {
-                        static_cast<__nv_bfloat16*>(p.out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(v);
+            for (int g = 0; g < WG; ++g) {
+                const int n = (nt * WG + g) * 128 + wrow;
+                if (n >= p.N) continue;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = 16 * h + i;
+                    if (m < p.M) {
+                        const float v = KIND == 1 ? __fmul_rn(acc[g][i], alpha) : acc[g][i];
+                        if constexpr (OUT_F32) {
+                            static_cast<float*>(p.out)[static_cast<int64_t>(m) * p.N + n] = v;
+                        } else {
+                            static_cast<__nv_bfloat16*>(p.out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(v);
+                        }
                     }
                 }
             }
@@ -2009,14 +2045,14 @@ bool make_out_tok_map(CUtensorMap* m, void* base, int64_t M, int64_t N) {
            CUDA_SUCCESS;
 }
 
-template <int KIND, bool F32, int QRULE>
+template <int KIND, int WG, bool F32, int QRULE>
 int run_decode(const void* x, const void* B_q, GemmArgs args, int splits, cudaStream_t stream) {
-    using C = DecCfg<KIND>;
-    auto kern = gemm_decode_kernel<KIND, F32, QRULE>;
+    using C = DecCfg<KIND, WG>;
+    auto kern = gemm_decode_kernel<KIND, WG, F32, QRULE>;
     CUtensorMap tx, tw, to;
-    // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 32 rows; W codes 128 rows x 128 bytes
+    // x: bf16 rows of 2 K bytes in boxes of 128 bytes (64 elements) x 32 rows; W codes 128 WG rows x 128 bytes
     if (!make_map(&tx, x, 2 * static_cast<uint64_t>(args.K), args.M, C::TOK) ||
-        !make_map(&tw, B_q, args.K / C::EPB, args.N, 128))
+        !make_map(&tw, B_q, args.K / C::EPB, args.N, 128 * WG))
         return MXQ_ERR_CUDA;
     memset(&to, 0, sizeof(to));
     args.tma_store = 0;
@@ -2025,9 +2061,10 @@ int run_decode(const void* x, const void* B_q, GemmArgs args, int splits, cudaSt
         args.tma_store = 1;
     }
     args.m_tiles = 1;
-    args.n_tiles = static_cast<int>(ceil_div(args.N, 128));
+    args.n_tiles = static_cast<int>(ceil_div(args.N, 128 * WG));
     args.k_stages = static_cast<int>(ceil_div(args.K, C::BK));
     args.k_split = static_cast<uint32_t>(splits);
+    if (WG > 1 && splits != 1) return MXQ_ERR_UNSUPPORTED;  // two weight groups are never split along K
     int dev = 0;
     cudaGetDevice(&dev);
     static bool attr_done[64] = {};
@@ -2189,8 +2226,12 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
 namespace {
 template <int KIND, bool F32>
 int fused_rule(const void* W_q, const GemmArgs& a, int rule, int splits, cudaStream_t stream) {
-    return rule == MXQ_RULE_CEIL ? run_decode<KIND, F32, MXQ_RULE_CEIL>(a.x, W_q, a, splits, stream)
-                                 : run_decode<KIND, F32, MXQ_RULE_EVEN>(a.x, W_q, a, splits, stream);
+    if (splits >= 2)  // 128 weight rows per CTA, K split over a cluster
+        return rule == MXQ_RULE_CEIL ? run_decode<KIND, 1, F32, MXQ_RULE_CEIL>(a.x, W_q, a, splits, stream)
+                                     : run_decode<KIND, 1, F32, MXQ_RULE_EVEN>(a.x, W_q, a, splits, stream);
+    // many weight rows: 256 per CTA, no K split
+    return rule == MXQ_RULE_CEIL ? run_decode<KIND, 2, F32, MXQ_RULE_CEIL>(a.x, W_q, a, 1, stream)
+                                 : run_decode<KIND, 2, F32, MXQ_RULE_EVEN>(a.x, W_q, a, 1, stream);
 }
 template <int KIND, bool F32>
 int rowq_rule(const void* x, const void* W_q, const GemmArgs& a, int rule, int splits, cudaStream_t stream) {
@@ -2205,11 +2246,14 @@ bool rowq_applies(int64_t M, int64_t N) { return M > 32 && N <= RowqCfg<0>::BN; 
 
 int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt) {
     if (rowq_applies(M, N)) return rowq_splits(M, K, fmt == MXQ_MXFP8 ? RowqCfg<2>::BK : RowqCfg<0>::BK);
-    // the bf16 activations of a stage (rows rounded up to 8, BK elements) must fit the A buffer
+    // up to 32 tokens: the few-token kernel, with 128 weight rows per CTA and a K split where that
+    // fills the SMs, else with 256 weight rows per CTA where those tiles fit one wave; with more
+    // weight rows than that, the quantizer and the persistent GEMM
     if (M > 32) return 0;
     const int bk = fmt == MXQ_MXFP8 ? Cfg<2, 128, 6>::BK : Cfg<0, 128, 6>::BK;
     const int splits = splitk_count(N, K, bk);
-    return splits < 2 ? 0 : splits;
+    if (splits >= 2) return splits;
+    return ceil_div(N, 256) <= sm_count() ? 1 : 0;
 }
 
 int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, const float* g_W, const float* g_A,
@@ -2217,7 +2261,7 @@ int launch_linear_fused(const void* x, const void* W_q, const uint8_t* W_sf, con
                         cudaStream_t stream) {
     const int splits = linear_fused_splits(M, N, K, fmt);
     const bool rowq = rowq_applies(M, N);
-    if (!rowq && splits < 2) return kNotFused;
+    if (!rowq && splits < 1) return kNotFused;
     GemmArgs a = {};
     a.x = x;
     a.b_sf = W_sf;

@@ -66,12 +66,12 @@ int launch_gemm(const void* A_q, const uint8_t* A_sf, const void* B_q, const uin
                 cudaStream_t stream, bool pdl_secondary);
 
 // Linear layer in one launch where the GEMM quantizes the bf16 activations x itself (rule `rule`
-// for MX formats, global scale g_A for NVFP4) with the quantizer's arithmetic: the split-K GEMM for
-// up to 32 tokens with several K splits (the result equals quantize-then-GEMM bit for bit), and the
-// small-N kernel for more tokens and N <= 128.  Returns kNotFused (nothing launched) otherwise;
-// arguments already validated.
+// for MX formats, global scale g_A for NVFP4) with the quantizer's arithmetic: the few-token kernel
+// for up to 32 tokens (the result equals quantize-then-GEMM bit for bit), and the small-N kernel
+// for more tokens and N <= 128.  Returns kNotFused (nothing launched) otherwise; arguments already
+// validated.
 constexpr int kNotFused = 1;
-// K splits of the one-launch path for this problem on the current device (the split-K GEMM
+// K splits of the one-launch path for this problem on the current device (the few-token kernel
 // quantizing up to 32 token rows, or the small-N kernel quantizing whole 128-row M tiles for N <= 128;
 // 1 when that kernel runs without a K split), 0 when no one-launch path applies.
 int linear_fused_splits(int64_t M, int64_t N, int64_t K, int fmt);

@@ -139,12 +139,14 @@ def test_linear_matches_oracle(fmt, M, N, K):
 @pytest.mark.parametrize("fmt,rule", [("mxfp4", "ceil"), ("mxfp4", "even"), ("nvfp4", "ceil"), ("mxfp8", "ceil"),
                                       ("mxfp8", "even")])
 @pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (32, 512, 2048), (17, 300, 320), (7, 96, 5120), (100, 300, 320),
-                                   (128, 640, 768)])
+                                   (128, 640, 768), (9, 33000, 320), (1, 20001, 256)])
 def test_linear_one_launch_equals_quantize_then_gemm(fmt, rule, M, N, K):
     """Up to 32 tokens: mxq_linear's GEMM quantizes the activations itself (one launch).  Its output
     equals quantizing with mxq_quantize and multiplying with mxq_gemm, bit for bit, including a K
     tail that leaves the last stage partly empty (K = 320), ragged and single-token problems; the
-    M = 100 and 128 cases take the two-launch path."""
+    M = 100 and 128 cases take the two-launch path.  N = 33000 and 20001 have more weight tiles
+    than K splits can use: 256 weight rows per CTA, no K split, a last tile that is partly (N =
+    33000) or half (N = 20001, also not a multiple of 8: direct stores) past N."""
     if fmt == "mxfp8" and K % 32:
         pytest.skip("K")
     A = synth.random_bf16((M, K), 7 + M + K, std=1.0).cuda()
@@ -206,7 +208,8 @@ def test_linear_kernel_count():
     assert mxq.linear_kernel_count(7, 96, 5120, "mxfp8") == 1
     assert mxq.linear_kernel_count(100, 300, 320, "mxfp4") == 2
     assert mxq.linear_kernel_count(8192, 34816, 5120, "mxfp4") == 2
-    assert mxq.linear_kernel_count(32, 34816, 5120, "mxfp4") == 2  # one K split: quantizer + GEMM
+    assert mxq.linear_kernel_count(32, 34816, 5120, "mxfp4") == 1  # 256 weight rows per CTA, one wave
+    assert mxq.linear_kernel_count(32, 151936, 5120, "mxfp4") == 2  # more than one wave: quantizer + GEMM
     assert mxq.linear_kernel_count(8192, 96, 5120, "mxfp8") == 1  # small N: the GEMM quantizes its rows
     assert mxq.linear_kernel_count(8192, 129, 5120, "mxfp8") == 2
 
