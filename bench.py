@@ -267,37 +267,54 @@ def run_mxq(args, world, rank, local):
     mxq.mxq_device_status(reset=True)
 
     timing = "eager calls through the binding"
+
+    def run_steps(n):
+        for _ in range(n):
+            step()
+
     if M <= 32:
         # few tokens: a call is a few microseconds of GPU work, less than the host needs to launch it
-        # through the Python binding (about 12 us), so each step replays a CUDA graph holding that
-        # step's call (one graph per weight copy), as serving replays its decode steps; the host's
-        # launch cost stays outside the measurement
+        # through the Python binding (about 12 us) or to replay a one-call CUDA graph (about 2.5 us of
+        # launch gap per replay), so the steps run from CUDA graphs of consecutive calls, each call on
+        # the next weight copy, as serving replays one graph over a decode step's layers; every step
+        # is still one full call (its own weights from HBM, its activations quantized, its output stored)
         gs = torch.cuda.Stream(device=dev)
-        graphs = []
         torch.cuda.synchronize()
-        for wq, wsf in wset:
+
+        def capture(n):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=gs):
-                mxq.linear(A, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
-                           workspace=ws, out=out)
-            graphs.append(g)
+                for i in range(n):
+                    wq, wsf = wset[i % copies]
+                    mxq.linear(A, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
+                               workspace=ws, out=out)
+            return g
 
-        def step():
-            graphs[it[0] % copies].replay()
-            it[0] += 1
+        per_graph = copies * -(-16 // copies)  # a whole number of weight-copy rotations, at least 16 calls
+        graphs = {per_graph: capture(per_graph)}
 
-        for _ in range(max(3, args.warmup)):
-            step()
+        def run_steps(n):
+            # exactly n calls: whole graphs of per_graph calls, then one graph of the remainder
+            for _ in range(n // per_graph):
+                graphs[per_graph].replay()
+            r = n % per_graph
+            if r:
+                if r not in graphs:
+                    graphs[r] = capture(r)
+                graphs[r].replay()
+
+        run_steps(max(3, args.warmup))
+        run_steps(args.steps % per_graph)  # capture the remainder graph outside the timed region
         torch.cuda.synchronize()
-        timing = "one CUDA graph replay per step (the host launch cost is outside the graph)"
+        timing = ("CUDA graphs of %d consecutive calls (each on the next weight copy), %d steps in all; the host "
+                  "launch cost stays outside the measurement" % (per_graph, args.steps))
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         start.record(stream)
-        for _ in range(args.steps):
-            step()
+        run_steps(args.steps)
         end.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -340,23 +357,29 @@ def run_mxq(args, world, rank, local):
         # linear call itself when that is one launch (the GEMM quantizing its own activations: bf16
         # rows in), else as the GEMM on quantized activations
         if one_launch:
+            # one launch per step: its average duration is the timed region's per step, with the
+            # weights streamed from HBM (rotating copies) or a working set larger than the L2
             lin_cold = time_flushed(lambda: mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype,
                                                        g_W=g_w, g_A=g_a, workspace=ws, out=out, stream=stream),
                                     20, stream, flush)
+            lin_s = elapsed / args.steps
             gbytes = W_q.numel() + W_sf.numel() + 2 * M * K + out.numel() * out.element_size()
             kname = ("gemm_decode_kernel (tcgen05 kind::%s, few tokens, activations quantized in the kernel)" if M <= 32
                      else "gemm_rowq_kernel (tcgen05 kind::%s, few columns, activations quantized in the kernel)") % kind
         else:
             lin_cold = time_flushed(lambda: mxq.gemm(a_q, a_sf, W_q, W_sf, M, N, K, fmt, out_dtype=out_dtype, g_A=g_a,
                                                      g_B=g_w, out=out, stream=stream), 20, stream, flush)
+            lin_s = lin_cold
             gbytes = W_q.numel() + W_sf.numel() + a_q.numel() + a_sf.numel() + out.numel() * out.element_size()
             kname = "gemm_splitk_kernel / gemm_kernel (tcgen05 kind::%s, few tokens)" % kind
         roofline = {"bound": "hbm", "kernel": kname,
-                    "achieved": round(gbytes / lin_cold / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
-                    "frac": round(gbytes / lin_cold / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
+                    "achieved": round(gbytes / lin_s / 1e9, 1), "peak": round(hbm_gbs, 1), "unit": "GB/s",
+                    "frac": round(gbytes / lin_s / 1e9 / hbm_gbs, 4), "peak_source": "%s HBM copy" % peak_src,
                     "traffic": traffic_for("linear_%s_%s" % (fmt, workload)) if one_launch else None,
-                    "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(lin_cold * 1e3, 4),
-                    "l2": "flushed per launch (the launch latency is inside the time)"}
+                    "algorithmic_bytes_per_launch": gbytes, "ms_per_launch": round(lin_s * 1e3, 4),
+                    "l2": ("average launch over the timed region (%s)" % l2_note if one_launch else
+                           "flushed per launch (the launch latency is inside the time)"),
+                    "ms_single_launch_l2_flushed": round(lin_cold * 1e3, 4)}
     qb = QUANT_BYTES_PER_ELEM[fmt] * M * K
     quant = {"workload": "activation quantize %dx%d %s %s" % (M, K, fmt, cfg["a_rule"]),
              "gbs": round(qb / quant_s / 1e9, 1), "frac": round(qb / quant_s / 1e9 / hbm_gbs, 4),
@@ -446,25 +469,28 @@ def other_workloads(stream, bf16_tflops):
             del q, sf, flush
         for _ in range(3):
             f()
-        if M <= 32:  # few tokens: replay a graph of the call, as for the decode bench (host launch cost outside)
+        calls = 1
+        if M <= 32:  # few tokens: graphs of 16 calls, as for the decode bench (host launch cost outside)
+            calls = 16
             gs = torch.cuda.Stream()
             torch.cuda.synchronize()
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=gs):
-                mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], g_W=g_w, g_A=g_a, workspace=ws, out=out)
+                for _ in range(calls):
+                    mxq.linear(A, W_q, W_sf, N, fmt, act_rule=cfg["a_rule"], g_W=g_w, g_A=g_a, workspace=ws, out=out)
             f = gr.replay
             for _ in range(3):
                 f()
         iters = 200 if M * N < 1e8 else 30
-        t = time_loop(f, iters, stream)
+        t = time_loop(f, max(1, iters // calls), stream) / calls
         peak = bf16_tflops * (FP8_PER_BF16 if fmt == "mxfp8" else FP4_PER_BF16)
         r = {"M": M, "N": N, "K": K, "fmt": fmt, "ms": round(t * 1e3, 4), "tflops": round(2.0 * M * N * K / t / 1e12, 1),
              "frac_of_measured_peak": round(2.0 * M * N * K / t / 1e12 / peak, 4)}
         if name == "decode":  # weight-stream bound: codes + scales of W per call
             wbytes = W_q.numel() + W_sf.numel()
             r["weight_gbs"] = round(wbytes / t / 1e9, 1)
-            r["l2"] = ("back-to-back CUDA graph replays of the call on one weight copy (L2-resident); --workload decode "
-                       "streams them from HBM")
+            r["l2"] = ("CUDA graphs of 16 calls on one weight copy (L2-resident); --workload decode streams them from "
+                       "HBM")
         r.update(qr)
         res[name] = r
         del A, W_q, W_sf, ws, out
@@ -481,22 +507,25 @@ def other_workloads(stream, bf16_tflops):
         f = lambda: mxq.gemm_w4a16(A, W_q, W_sf, N, "mxfp4", out=out, stream=stream)
         for _ in range(3):
             f()
-        if M <= 32:  # few tokens: replay a graph of the call (host launch cost outside)
+        calls = 1
+        if M <= 32:  # few tokens: graphs of 16 calls (host launch cost outside)
+            calls = 16
             gs = torch.cuda.Stream()
             torch.cuda.synchronize()
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=gs):
-                mxq.gemm_w4a16(A, W_q, W_sf, N, "mxfp4", out=out)
+                for _ in range(calls):
+                    mxq.gemm_w4a16(A, W_q, W_sf, N, "mxfp4", out=out)
             f = gr.replay
             for _ in range(3):
                 f()
-        t = time_loop(f, 200 if M * N < 1e8 else 10, stream)
+        t = time_loop(f, max(1, (200 if M * N < 1e8 else 10) // calls), stream) / calls
         r = {"M": M, "N": N, "K": K, "fmt": "mxfp4 weights, bf16 activations", "ms": round(t * 1e3, 4),
              "tflops": round(2.0 * M * N * K / t / 1e12, 1),
              "frac_of_measured_bf16": round(2.0 * M * N * K / t / 1e12 / bf16_tflops, 4)}
         if name == "decode":
             r["weight_gbs"] = round((W_q.numel() + W_sf.numel()) / t / 1e9, 1)
-            r["l2"] = "back-to-back CUDA graph replays on one weight copy (L2-resident)"
+            r["l2"] = "CUDA graphs of 16 calls on one weight copy (L2-resident)"
         res["w4a16_" + name] = r
         del A, W_q, W_sf, out
         torch.cuda.empty_cache()

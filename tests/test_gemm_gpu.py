@@ -166,6 +166,32 @@ def test_linear_one_launch_equals_quantize_then_gemm(fmt, rule, M, N, K):
     assert mxq.mxq_device_status(reset=True) == 0
 
 
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("M,N,K", [(32, 512, 2048), (5, 33000, 320)])
+def test_linear_one_launch_x_16_byte_aligned(fmt, M, N, K):
+    """The API promises 16-byte alignment of x, which is all the few-token kernel's 16-byte token
+    loads need.  x here starts 16 bytes into an allocation (not 32-byte aligned); the output equals
+    mxq_quantize + mxq_gemm bit for bit, and the same call on an aligned copy of x."""
+    base = synth.random_bf16((M * K + 8,), 11 + M + K, std=1.0).cuda()
+    A = base[8:].view(M, K)
+    assert A.data_ptr() % 32 == 16
+    W = synth.random_bf16((N, K), 12 + N, std=0.02).cuda()
+    g_w = g_a = None
+    if fmt == "nvfp4":
+        g_w, _ = mxq.global_scale(W)
+        g_a, _ = mxq.global_scale(A)
+    Wq, Wsf = mxq.quantize(W, fmt, "even", global_scale=g_w)
+    Aq, Asf = mxq.quantize(A, fmt, "ceil", global_scale=g_a)
+    two = mxq.gemm(Aq, Asf, Wq, Wsf, M, N, K, fmt, out_dtype=torch.float32, g_A=g_a, g_B=g_w)
+    one = mxq.linear(A, Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=torch.float32, g_W=g_w, g_A=g_a)
+    aligned = mxq.linear(A.clone(), Wq, Wsf, N, fmt, act_rule="ceil", out_dtype=torch.float32, g_W=g_w, g_A=g_a)
+    torch.cuda.synchronize()
+    assert mxq.linear_kernel_count(M, N, K, fmt) == 1
+    assert torch.equal(one.view(torch.int32), two.view(torch.int32))
+    assert torch.equal(one.view(torch.int32), aligned.view(torch.int32))
+    assert mxq.mxq_device_status(reset=True) == 0
+
+
 @pytest.mark.parametrize("fmt,rule", [("mxfp4", "ceil"), ("mxfp4", "even"), ("nvfp4", "even"), ("mxfp8", "even"),
                                       ("mxfp8", "ceil")])
 @pytest.mark.parametrize("M,N,K", [(33, 96, 512), (129, 1, 640), (300, 128, 320), (1000, 100, 1024), (257, 17, 5120),
