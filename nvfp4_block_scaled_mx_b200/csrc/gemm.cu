@@ -1490,10 +1490,17 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
 // A rows [128 r, +128) and B rows [BN/2 r, +BN/2) of the tile, so each SM streams 128 rows of A
 // and BN/2 rows of B per 128-byte K slice.  Every load of both CTAs (operands, the CTA's own A
 // scale tiles and the scale tiles of all the tile's B rows) is a TMA load that completes on the
-// leader's barrier; a scale warp in the leader then copies both CTAs' scale tiles into their TMEM
-// (tcgen05.cp.cta_group::2, each CTA from its own shared memory) and commits to a local barrier,
-// and the MMA warp issues the MMAs.  The only cross-CTA signals per stage are the TMA completions
-// and the MMA commit multicast to both CTAs.
+// leader's barrier; the leader's MMA warp then copies both CTAs' scale tiles into their TMEM
+// (tcgen05.cp.cta_group::2, each CTA from its own shared memory) and issues the stage's MMAs
+// behind them in the tensor pipe.  The only cross-CTA signals per stage are the TMA completions
+// and the MMA commit multicast to both CTAs.  (A separate scale-copy warp with a barrier of its
+// own put one more hop into every stage's round trip and measured 1-2 % slower.)
+//
+// A stage slot's round trip (reissued -> its data landed 1.5 us -> MMAs issued 0.2 us -> MMAs done
+// and the slot reissued 0.6 us) is about 2.2 us, with all SMs together pulling about 11.5 TB/s of
+// operands out of L2.  Without the operand loads the kernel runs at 6.9 PFLOP/s (MXFP4): each
+// block-scaled pair MMA costs about 0.085 us whether N is 256 or 128, so a 256 x 384 tile (an N =
+// 256 and an N = 128 MMA per K step, 17 % fewer operand bytes per FLOP) measured slower.
 //
 // BN = 256 keeps one accumulator (256 TMEM columns + the scale slots fill the 512), so the
 // tensor pipe idles while the epilogue drains it at every tile boundary.  BN = 192 fits two
@@ -1501,9 +1508,8 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
 // other.  A 192-row tile starts 0 or 64 rows into a 128-row scale tile; the MMA then addresses
 // the B scales 0 or 2 TMEM columns into the two copied scale tiles (32 rows per column).
 //   warp 0       TMA producer (both CTAs)
-//   warp 1       TMEM owner (both CTAs); MMA issuer (leader)
-//   warp 2       scale copies into TMEM (leader)
-//   warps 3-     epilogue (both CTAs): EPI_WARPS / 4 warps per TMEM sub-partition, COLS columns each
+//   warp 1       TMEM owner (both CTAs); scale copies and MMA issuer (leader)
+//   warps 2-     epilogue (both CTAs): EPI_WARPS / 4 warps per TMEM sub-partition, COLS columns each
 // The single-thread roles run as converged warps that issue through one elected lane.
 
 template <int KIND, int STAGES, int BN>
@@ -1518,7 +1524,7 @@ struct PairCfg {
     static constexpr int B_ROWS = BN / 2;              // B rows per CTA
     static constexpr int COLS = (BN == 256) ? 128 : 64;  // accumulator columns per epilogue warp
     static constexpr int EPI_WARPS = 4 * (BN / COLS);
-    static constexpr int THREADS = (3 + EPI_WARPS) * 32;
+    static constexpr int THREADS = (2 + EPI_WARPS) * 32;
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int SFA_BYTES = SF_ATOMS * 512;
@@ -1540,7 +1546,7 @@ struct PairCfg {
     static constexpr int STG_BYTES = 4096;
     static constexpr int OFF_STG = ((OFF_SFB + STAGES * SFB_BYTES) + 1023) / 1024 * 1024;
     static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
-    static constexpr int N_BARS = 3 * STAGES + 2 * ACC;
+    static constexpr int N_BARS = 2 * STAGES + 2 * ACC;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -1555,8 +1561,7 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // leader: all loads of both CTAs landed
-    uint64_t* sfready = full + STAGES;                                 // leader: scales copied into both TMEMs
-    uint64_t* empty = sfready + STAGES;                                // both: the stage's MMAs are done
+    uint64_t* empty = full + STAGES;                                   // both: the stage's MMAs are done
     uint64_t* accf = empty + STAGES;                                   // both: accumulator buffer ready
     uint64_t* acce = accf + C::ACC;                                    // leader: accumulator buffer drained by both
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_SLOT);
@@ -1571,7 +1576,6 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
         prefetch_tmap(&tma_sfb);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sfready[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < C::ACC; ++a) {
@@ -1651,7 +1655,7 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait_warp(&sfready[stage], phase, p.status, 13)) {
+                    if (!mbar_wait_warp(&full[stage], phase, p.status, 13)) {
                         ok = false;
                         break;
                     }
@@ -1659,7 +1663,19 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
                     const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
                     const uint32_t a_s = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
                     const uint32_t b_s = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
+                    const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
                     if (elect_one()) {
+                        // this stage's scale tiles into both CTAs' TMEM, ahead of its MMAs in the
+                        // tensor pipe (the slot's previous MMAs completed before its loads were issued)
+#pragma unroll
+                        for (int a = 0; a < C::SF_ATOMS; ++a) {
+                            tc_cp_scales_pair(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
+#pragma unroll
+                            for (int g = 0; g < 2; ++g)
+                                tc_cp_scales_pair(sf_col + C::SF_COLS_A + a * 8 + g * 4,
+                                                  smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
+                        }
 #pragma unroll
                         for (int j = 0; j < C::KSTEPS; ++j) {
                             if (ks * C::BK + j * C::MMA_K < p.K) {
@@ -1689,45 +1705,10 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
                 }
             }
         }
-    } else if (warp == 2) {
-        if (rank == 0) {
-            // scale copies into both CTAs' TMEM (leader): the whole warp runs the loop; one elected lane issues
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                for (int ks = 0; ks < p.k_stages; ++ks) {
-                    if (!mbar_wait_warp(&full[stage], phase, p.status, 16)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sf_col = tmem_base + C::SF_TMEM_BASE + stage * C::SF_COLS_STAGE;
-                    const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
-                    if (elect_one()) {
-#pragma unroll
-                        for (int a = 0; a < C::SF_ATOMS; ++a) {
-                            tc_cp_scales_pair(sf_col + a * 4, smem_desc(sfa_s + a * 512, 0, 128, kLayoutNone));
-#pragma unroll
-                            for (int g = 0; g < 2; ++g)
-                                tc_cp_scales_pair(sf_col + C::SF_COLS_A + a * 8 + g * 4,
-                                                  smem_desc(sfb_s + (g * C::SF_ATOMS + a) * 512, 0, 128, kLayoutNone));
-                        }
-                        tc_commit_pair(&sfready[stage], 0x1);
-                    }
-                    __syncwarp();
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-        }
     } else {
         constexpr int COLS = C::COLS;  // accumulator columns owned by this warp
         const int sub = warp & 3;
-        const int col0 = ((warp - 3) >> 2) * COLS;
+        const int col0 = ((warp - 2) >> 2) * COLS;
         const int row = sub * 32 + lane;
         const float alpha = (KIND == 1) ? __fmul_rn(*p.g_a, *p.g_b) : 1.0f;
         int acc = 0;
@@ -1776,7 +1757,7 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
                 if (p.tma_store) {
                     // 64 columns at a time: rows into the warp's 128B-swizzled staging tile, then one
                     // TMA store (clipped at the M / N edges), so the output leaves in full lines
-                    uint8_t* stg = smem + C::OFF_STG + (warp - 3) * C::STG_BYTES;
+                    uint8_t* stg = smem + C::OFF_STG + (warp - 2) * C::STG_BYTES;
 #pragma unroll
                     for (int h = 0; h < COLS / 64; ++h) {
                         if (lane == 0) bulk_wait_group_read0();
@@ -1849,7 +1830,7 @@ __global__ void __launch_bounds__(PairCfg<KIND, STAGES, BN>::THREADS, 1)
         }
     }
 
-    if (warp >= 3 && lane == 0) bulk_wait_group0();  // output stores of this warp have landed
+    if (warp >= 2 && lane == 0) bulk_wait_group0();  // output stores of this warp have landed
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // no CTA leaves while its peer may still signal its barriers or use its TMEM
@@ -2178,11 +2159,10 @@ int splitk_count(int64_t N, int64_t K, int bk) {
 
 template <int KIND, bool F32>
 int dispatch_bn(const void* A_q, const void* B_q, const GemmArgs& args, cudaStream_t stream, bool pdl) {
-    // More than 128 rows: CTA pairs on 256 x 256 tiles.  Up to 128 rows (decode): one CTA per
-    // 128 x 128 tile, which gives the most CTAs for the weight stream.
-    // 256 x 256 pair tiles with one accumulator.  256 x 192 tiles with two accumulators (BN = 192)
-    // remove the drain bubble at tile boundaries but measured slower on the prefill problems: at
-    // 384 tensor-pipe cycles per stage the MMA and scale-copy warps can no longer issue ahead.
+    // More than 128 rows: CTA pairs on 256 x 256 tiles with one accumulator.  Up to 128 rows
+    // (decode): one CTA per 128 x 128 tile, which gives the most CTAs for the weight stream.
+    // 256 x 192 tiles with two accumulators (BN = 192) remove the drain bubble at tile boundaries
+    // but measured slower on the prefill problems.
     if (args.M > 128) return run_pair<KIND, 5, 256, F32>(A_q, B_q, args, stream, pdl);
     const int splits = splitk_count(args.N, args.K, Cfg<KIND, 128, 6>::BK);
     if (splits > 1) return run_splitk<KIND, F32>(A_q, B_q, args, splits, stream, pdl);
