@@ -242,23 +242,35 @@ def run_mxq(args, world, rank, local):
     out_dtype = torch.float32 if cfg["out"] == "fp32" else torch.bfloat16
     out = torch.empty(M, N, dtype=out_dtype, device=dev)
     flops = 2.0 * M * N * K
-    # a working set smaller than the L2 (decode): consecutive steps read different copies of the
-    # weights (together more than twice the L2), as consecutive layers of a model do, so every step
-    # streams its weights from HBM; the activations stay L2-resident, as a previous layer leaves them
+    # a working set smaller than the L2: consecutive steps read different copies of the larger
+    # operand (together more than twice the L2) -- the weights at decode, as consecutive layers of a
+    # model do (the activations stay L2-resident, as a previous layer leaves them), the bf16
+    # activations of a few-column layer -- so that every step streams it from HBM
     L2_BYTES = 126 << 20
     wbytes = W_q.numel() + W_sf.numel()
-    working = wbytes + A.numel() * A.element_size() + out.numel() * out.element_size()
-    copies = 1 if working > L2_BYTES else -(-2 * L2_BYTES // wbytes)
-    wset = [(W_q, W_sf)] + [(W_q.clone(), W_sf.clone()) for _ in range(copies - 1)]
-    l2_note = ("working set > 126 MB L2, no flush" if copies == 1 else
-               "weights rotate through %d copies (%.0f MB > 2 x L2) between steps; activations L2-resident" % (
-                   copies, copies * wbytes / 1e6))
+    abytes = A.numel() * A.element_size()
+    working = wbytes + abytes + out.numel() * out.element_size()
+    rotate_a = working <= L2_BYTES and abytes > wbytes
+    copies = 1 if working > L2_BYTES else -(-2 * L2_BYTES // (abytes if rotate_a else wbytes))
+    wset = [(W_q, W_sf)] + ([] if rotate_a else [(W_q.clone(), W_sf.clone()) for _ in range(copies - 1)])
+    aset = [A] + ([A.clone() for _ in range(copies - 1)] if rotate_a else [])
+    if copies == 1:
+        l2_note = "working set > 126 MB L2, no flush"
+    elif rotate_a:
+        l2_note = ("bf16 activations rotate through %d copies (%.0f MB > 2 x L2) between steps; weights "
+                   "L2-resident" % (copies, copies * abytes / 1e6))
+    else:
+        l2_note = ("weights rotate through %d copies (%.0f MB > 2 x L2) between steps; activations L2-resident" % (
+            copies, copies * wbytes / 1e6))
     it = [0]
 
+    def operands(i):
+        return aset[i % len(aset)], wset[i % len(wset)]
+
     def step():
-        wq, wsf = wset[it[0] % copies]
+        x, (wq, wsf) = operands(it[0])
         it[0] += 1
-        mxq.linear(A, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
+        mxq.linear(x, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
                    workspace=ws, out=out, stream=stream)
 
     for _ in range(max(3, args.warmup)):
@@ -272,12 +284,14 @@ def run_mxq(args, world, rank, local):
         for _ in range(n):
             step()
 
-    if M <= 32:
-        # few tokens: a call is a few microseconds of GPU work, less than the host needs to launch it
-        # through the Python binding (about 12 us) or to replay a one-call CUDA graph (about 2.5 us of
-        # launch gap per replay), so the steps run from CUDA graphs of consecutive calls, each call on
-        # the next weight copy, as serving replays one graph over a decode step's layers; every step
-        # is still one full call (its own weights from HBM, its activations quantized, its output stored)
+    one_launch = mxq.linear_kernel_count(M, N, K, fmt) == 1
+    if one_launch:
+        # one launch per call (few tokens, or few columns): a call is microseconds of GPU work, not
+        # much more than the host needs to launch it through the Python binding (about 12 us) or to
+        # replay a one-call CUDA graph (about 2.5 us of launch gap per replay), so the steps run from
+        # CUDA graphs of consecutive calls, each call on the next operand copy, as serving replays
+        # one graph over a step's layers; every step is still one full call (its operands from HBM,
+        # its activations quantized, its output stored)
         gs = torch.cuda.Stream(device=dev)
         torch.cuda.synchronize()
 
@@ -285,8 +299,8 @@ def run_mxq(args, world, rank, local):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=gs):
                 for i in range(n):
-                    wq, wsf = wset[i % copies]
-                    mxq.linear(A, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
+                    x, (wq, wsf) = operands(i)
+                    mxq.linear(x, wq, wsf, N, fmt, act_rule=cfg["a_rule"], out_dtype=out_dtype, g_W=g_w, g_A=g_a,
                                workspace=ws, out=out)
             return g
 
@@ -306,7 +320,7 @@ def run_mxq(args, world, rank, local):
         run_steps(max(3, args.warmup))
         run_steps(args.steps % per_graph)  # capture the remainder graph outside the timed region
         torch.cuda.synchronize()
-        timing = ("CUDA graphs of %d consecutive calls (each on the next weight copy), %d steps in all; the host "
+        timing = ("CUDA graphs of %d consecutive calls (each on the next operand copy), %d steps in all; the host "
                   "launch cost stays outside the measurement" % (per_graph, args.steps))
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -350,7 +364,6 @@ def run_mxq(args, world, rank, local):
                                            if sustained_bf16_tflops() else None),
                 "traffic": traffic_for("gemm_%s_%s" % (fmt, workload)),
                 "algorithmic_flops_per_launch": flops, "ms_per_launch": round(gemm_s * 1e3, 4)}
-    one_launch = mxq.linear_kernel_count(M, N, K, fmt) == 1
     if M <= 128 or one_launch:
         # few tokens or few columns: the layer streams its weights (few tokens) or its bf16 activations
         # (few columns) once and is HBM-bound.  Timed with the L2 flushed before each launch, as the
@@ -491,6 +504,9 @@ def other_workloads(stream, bf16_tflops):
             r["weight_gbs"] = round(wbytes / t / 1e9, 1)
             r["l2"] = ("CUDA graphs of 16 calls on one weight copy (L2-resident); --workload decode streams them from "
                        "HBM")
+        if name == "in_proj_ba":
+            r["l2"] = ("back-to-back eager calls on one activation tensor (84 MB, partly L2-resident); --workload "
+                       "in_proj_ba streams rotating copies from HBM")
         r.update(qr)
         res[name] = r
         del A, W_q, W_sf, ws, out

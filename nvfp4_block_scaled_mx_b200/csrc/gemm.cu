@@ -1112,7 +1112,8 @@ struct RowqCfg {
     static constexpr int SF_ATOMS = BK / BS / 4;  // 512-byte scale tiles per 128 rows per stage
     static constexpr int BN = 128;
     static constexpr int XSLOTS = 8;              // bf16 slots of 64 elements x 128 rows
-    static constexpr int XPS = BK / 64;           // slots per stage (4 FP4, 2 MXFP8)
+    static constexpr int XPS = BK / 64;           // slots per stage (4 FP4, 2 MXFP8), one barrier per stage
+    static constexpr int XSTAGES = XSLOTS / XPS;
     static constexpr int ASTAGES = 2, BSTAGES = 2;
     static constexpr int X_BYTES = 128 * 128;
     static constexpr int A_BYTES = 128 * 128;
@@ -1127,7 +1128,7 @@ struct RowqCfg {
     static constexpr int OFF_SFB = OFF_SFA + ASTAGES * SF_BYTES;
     static constexpr int OFF_TAB = OFF_SFB + BSTAGES * SF_BYTES;  // NVFP4 d and 1/d per scale code
     static constexpr int OFF_BAR = OFF_TAB + 1024;
-    static constexpr int N_BARS = 2 * (XSLOTS + ASTAGES + BSTAGES) + 3;  // + accf, rready, rfull
+    static constexpr int N_BARS = 2 * (XSTAGES + ASTAGES + BSTAGES) + 3;  // + accf, rready, rfull
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
     static constexpr int SLOT_COLS = 2 * SF_ATOMS * 4;  // per B stage: A then B scale tiles
@@ -1147,12 +1148,12 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     gemm_rowq_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_out, const GemmArgs p) {
     using C = RowqCfg<KIND>;
-    constexpr int BN = C::BN, XS = C::XSLOTS, AS = C::ASTAGES, BSt = C::BSTAGES;
+    constexpr int BN = C::BN, AS = C::ASTAGES, BSt = C::BSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* xempty = xfull + XS;
-    uint64_t* aready = xempty + XS;
+    uint64_t* xempty = xfull + C::XSTAGES;
+    uint64_t* aready = xempty + C::XSTAGES;
     uint64_t* aempty = aready + AS;
     uint64_t* bfull = aempty + AS;
     uint64_t* bempty = bfull + BSt;
@@ -1174,7 +1175,7 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tma_x);
         prefetch_tmap(&tma_b);
-        for (int s = 0; s < XS; ++s) {
+        for (int s = 0; s < C::XSTAGES; ++s) {
             mbar_init(&xfull[s], 1);
             mbar_init(&xempty[s], C::QWARPS);
         }
@@ -1207,26 +1208,25 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     pdl_launch_dependents();  // the next kernel on the stream may start its prologue
 
     if (warp == 0) {
-        // bf16 producer: slot (stage - k0) * XPS + b, b the 64-element box of the stage
+        // bf16 producer: the XPS 64-element boxes of a stage land in slots xs * XPS + b and complete
+        // on one barrier (a barrier per box made this one thread's loads complete about one at a
+        // time, 0.5 us per 16 KB box from HBM)
         const uint64_t pol = policy_evict_first();
-        int slot = 0;
+        int xs = 0;
         uint32_t phase = 0;
         for (int ks = k0; ks < k1; ++ks) {
-            for (int b = 0; b < C::XPS; ++b) {
-                if (!mbar_wait_warp(&xempty[slot], phase ^ 1u, p.status, 41)) {
-                    ks = k1;
-                    break;
-                }
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(&xfull[slot], C::X_BYTES);
-                    tma_load_2d(&tma_x, &xfull[slot], smem + C::OFF_X + slot * C::X_BYTES, (ks * C::BK + b * 64) * 2,
-                                mt * 128, pol);
-                }
-                __syncwarp();
-                if (++slot == XS) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
+            if (!mbar_wait_warp(&xempty[xs], phase ^ 1u, p.status, 41)) break;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&xfull[xs], C::XPS * C::X_BYTES);
+#pragma unroll
+                for (int b = 0; b < C::XPS; ++b)
+                    tma_load_2d(&tma_x, &xfull[xs], smem + C::OFF_X + (xs * C::XPS + b) * C::X_BYTES,
+                                (ks * C::BK + b * 64) * 2, mt * 128, pol);
+            }
+            __syncwarp();
+            if (++xs == C::XSTAGES) {
+                xs = 0;
+                phase ^= 1u;
             }
         }
     } else if (warp == 2) {
@@ -1317,16 +1317,11 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
             }
             named_barrier_sync(1, 32 * C::QWARPS);
         }
-        int xslot = 0, as = 0;
+        int xs = 0, as = 0;
         uint32_t xph = 0, aph = 0;
         bool ok = true;
         for (int ks = k0; ks < k1 && ok; ++ks) {
-#pragma unroll
-            for (int b = 0; b < C::XPS; ++b) {
-                const int sl = (xslot + b) % XS;
-                const uint32_t ph = xph ^ static_cast<uint32_t>((xslot + b) / XS);
-                ok = ok && mbar_wait_warp(&xfull[sl], ph & 1u, p.status, 44);
-            }
+            ok = mbar_wait_warp(&xfull[xs], xph, p.status, 44);
             if (!ok || !mbar_wait_warp(&aempty[as], aph ^ 1u, p.status, 49)) break;
             const uint32_t a_s = smem_u32(smem + C::OFF_A + as * C::A_BYTES);
             uint8_t* sfa = smem + C::OFF_SFA + as * C::SF_BYTES;
@@ -1336,7 +1331,7 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
                 const int row = v & 127, j = v >> 7;
                 if (static_cast<int64_t>(ks) * C::BK + j * 32 >= p.K) continue;
                 uint32_t w[16];
-                const uint32_t rb = smem_u32(smem + C::OFF_X + ((xslot + (j >> 1)) % XS) * C::X_BYTES) + row * 128;
+                const uint32_t rb = smem_u32(smem + C::OFF_X + (xs * C::XPS + (j >> 1)) * C::X_BYTES) + row * 128;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint4 t = ld_shared_v4(rb + ((((j & 1) * 4 + i) ^ (row & 7)) << 4));
@@ -1367,12 +1362,10 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&aready[as]);
-#pragma unroll
-                for (int b = 0; b < C::XPS; ++b) mbar_arrive(&xempty[(xslot + b) % XS]);
+                mbar_arrive(&xempty[xs]);
             }
-            xslot += C::XPS;
-            if (xslot >= XS) {
-                xslot -= XS;
+            if (++xs == C::XSTAGES) {
+                xs = 0;
                 xph ^= 1u;
             }
             if (++as == AS) {
