@@ -119,10 +119,10 @@ struct GemmArgs {
     int b_row_tiles;   // ceil(N / 128)
     int m_tiles, n_tiles, k_stages;
     int* status;
-    uint32_t k_split;      // split-K kernel: CTAs per cluster sharing one output tile
+    uint32_t k_split;      // K-split kernels: CTAs per cluster sharing one output tile
     uint32_t a_box_bytes;  // split-K kernel: bytes of one A load (rows rounded up to 8, <= 128)
     uint32_t tma_store;    // pair kernel: bf16 output written through TMA stores (N % 8 == 0)
-    const void* x;         // split-K kernel quantizing its own A: the bf16 activations [M, K]
+    const void* x;         // few-token and small-N kernels, which quantize their own A: the bf16 activations [M, K]
     int group_m;           // pair kernel: M tiles per raster group (m_tiles: plain M-fastest order)
 };
 
@@ -2212,7 +2212,7 @@ int rowq_rule(const void* x, const void* W_q, const GemmArgs& a, int rule, int s
                                  : run_rowq<KIND, F32, MXQ_RULE_EVEN>(x, W_q, a, splits, stream);
 }
 
-// Few output columns and more tokens than the split-K kernel quantizes itself: one column tile, so
+// Few output columns and more tokens than the few-token kernel quantizes itself: one column tile, so
 // the small-N kernel reads each activation row once and quantizes it on the way in.
 bool rowq_applies(int64_t M, int64_t N) { return M > 32 && N <= RowqCfg<0>::BN; }
 }  // namespace
