@@ -471,13 +471,19 @@ struct W16TCfg {
     static constexpr int OFF_ACT = 0;
     static constexpr int OFF_W = OFF_ACT + STAGES * ACT_BYTES;
     static constexpr int OFF_SF = OFF_W + STAGES * W_BYTES;
-    static constexpr int OFF_BAR = OFF_SF + STAGES * SF_BYTES;
+    // SPLIT at NT = 32: the partials of up to 3 other CTAs (16 KB each) get a buffer of their own, so
+    // that the other CTAs send them as soon as their MMAs are done; otherwise (NT = 64, 32 KB each)
+    // they reuse the leader's operand ring once the leader signals that its MMAs are done
+    static constexpr bool RED_OWN = SPLIT && NT == 32;
+    static constexpr int OFF_RED = OFF_SF + STAGES * SF_BYTES;
+    static constexpr int RED_BYTES = RED_OWN ? 3 * 128 * NT * 4 : 0;
+    static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
     static constexpr int N_BARS = 2 * STAGES + 2 * AS + 2 * ACC + 2;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_SLOT + 16 + 1024;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N");
     static_assert(COLS_USED <= 512, "TMEM budget");
-    static_assert(!SPLIT || 3 * 128 * NT * 4 <= OFF_BAR, "split-K partials fit below the barriers");
+    static_assert(!SPLIT || RED_OWN || 3 * 128 * NT * 4 <= OFF_RED, "split-K partials fit in the operand ring");
     static_assert(ACT_SUB % 1024 == 0, "128B-swizzled activation boxes stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -794,18 +800,20 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         tc_fence_before();
         __syncthreads();
     } else {
-        // every CTA's epilogue warps take their partial tile into registers.  The leader frees its
-        // operand ring once its MMAs are done (a remote arrive per other CTA); the others send their
-        // partials with st.async, counted in bytes on the leader's barrier, and leave.  Layout in
+        // every CTA's epilogue warps take their partial tile into registers.  The others send their
+        // partials with st.async, counted in bytes on the leader's barrier, and leave: at NT = 32
+        // into a buffer of the leader's own at once (the hand-shake below cost about 0.9 us between
+        // the leader's last MMAs and the partials leaving), at NT = 64 into the leader's operand
+        // ring once the leader has freed it (a remote arrive per other CTA).  Layout in
         // the leader: [splits-1][NT/4 column quads][128 rows][4] fp32, so that the 32 rows of a warp
         // move 512 contiguous bytes per 16-byte access.
         float part[HC];
-        float* red = reinterpret_cast<float*>(smem);
+        float* red = reinterpret_cast<float*>(smem + (C::RED_OWN ? C::OFF_RED : 0));
         const int row = sub * 32 + lane;
         cluster_wait();  // every CTA of the cluster has initialised its barriers
         if (epi) {
             const bool ok = mbar_wait(&accf[0], 0, p.status, 58);
-            if (split == 0 && warp == 2 + kWtDeqWarps && lane == 0)
+            if (!C::RED_OWN && split == 0 && warp == 2 + kWtDeqWarps && lane == 0)
                 for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(half * HC);
@@ -819,7 +827,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
             }
             tc_fence_before();
         }
-        if (epi && split != 0 && mbar_wait_cluster(rready, 0, p.status, 59)) {
+        if (epi && split != 0 && (C::RED_OWN || mbar_wait_cluster(rready, 0, p.status, 59))) {
             const uint32_t dst =
                 mapa_shared(smem_u32(red + (((split - 1) * (NT / 4) + half * HC / 4) * 128 + row) * 4), 0);
             const uint32_t bar = mapa_shared(smem_u32(rfull), 0);
@@ -1069,7 +1077,7 @@ int dispatch_w16(const void* A, const void* Wq, const uint8_t* Wsf, const float*
                                    : run_w16t<FMT, 64, 4, 3, false, 8, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1);
     }
     const int s = w16_splits(w_tiles, k_stages, 4);
-    if (s > 1) return run_w16t<FMT, 32, 6, 3, true, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, s);
+    if (s > 1) return run_w16t<FMT, 32, 5, 3, true, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, s);
     return w_tiles <= sm_count() ? run_w16t<FMT, 32, 6, 3, false, 16, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1)
                                  : run_w16t<FMT, 32, 6, 3, false, 8, F32>(A, Wq, Wsf, g_w, M, N, K, out, stream, 1);
 }
