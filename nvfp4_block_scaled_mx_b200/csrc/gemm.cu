@@ -1139,6 +1139,8 @@ struct RowqCfg {
     static_assert(XSLOTS % XPS == 0, "whole stages in the bf16 ring");
     static_assert(SF_TMEM_BASE + BSTAGES * SLOT_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
     static_assert((kMaxSplits - 1) * 128 * BN * 4 <= OFF_TAB, "reduction buffer inside the rings");
+    static constexpr int EARLY_SPLITS = XSLOTS * X_BYTES / (128 * BN * 4) + 1;  // partials inside the bf16 ring
+    static_assert(EARLY_SPLITS >= 2, "at least one partial fits in the bf16 ring");
     static_assert(QWARPS * STG_BYTES <= OFF_TAB, "output staging inside the rings");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -1373,10 +1375,19 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
                 aph ^= 1u;
             }
         }
+        // with up to EARLY_SPLITS CTAs the partials land in the leader's bf16 ring only, which is
+        // idle once every quantizer warp is done with the last stage: the leader lets the other
+        // CTAs send them now, while its last MMAs still run, instead of after them
+        if (split == 0 && splits > 1 && splits <= static_cast<uint32_t>(C::EARLY_SPLITS)) {
+            named_barrier_sync(3, 32 * C::QWARPS);
+            if (warp == 3 && lane == 0)
+                for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
+        }
     }
 
     // reduction and epilogue: warps 3-18 hold 32 accumulator columns of one TMEM sub-partition
-    // each; the leader frees its rings for the partials once its MMAs are done, the others send
+    // each; the leader frees its rings for the partials (its bf16 ring once its quantizers are done
+    // with it, for up to EARLY_SPLITS CTAs; else its rings once its MMAs are done), the others send
     // their valid rows with st.async (column-quad-major layout, as in the split-K kernel) and
     // leave; the leader adds them in split order and stores through a staging tile per warp and a
     // TMA store (rows per lane, so direct stores would touch one sector per element)
@@ -1390,7 +1401,7 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     cluster_wait();  // every CTA of the cluster has initialised its barriers
     if (epi) {
         const bool ok = mbar_wait(accf, 0, p.status, 45);
-        if (split == 0 && warp == 3 && lane == 0)
+        if (split == 0 && splits > static_cast<uint32_t>(C::EARLY_SPLITS) && warp == 3 && lane == 0)
             for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
         tc_fence_after();
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(col0);
