@@ -1379,6 +1379,7 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
         // idle once every quantizer warp is done with the last stage: the leader lets the other
         // CTAs send them now, while its last MMAs still run, instead of after them
         if (split == 0 && splits > 1 && splits <= static_cast<uint32_t>(C::EARLY_SPLITS)) {
+            cluster_wait();  // the other CTAs' barriers are initialised (these warps wait here, not below)
             named_barrier_sync(3, 32 * C::QWARPS);
             if (warp == 3 && lane == 0)
                 for (uint32_t sp = 1; sp < splits; ++sp) mbar_arrive_cluster(mapa_shared(smem_u32(rready), sp));
@@ -1398,7 +1399,8 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
     const int row = sub * 32 + lane;
     float* red = reinterpret_cast<float*>(smem);
     float acc[COLS];
-    cluster_wait();  // every CTA of the cluster has initialised its barriers
+    const bool early = split == 0 && splits > 1 && splits <= static_cast<uint32_t>(C::EARLY_SPLITS);
+    if (!(epi && early)) cluster_wait();  // every CTA of the cluster has initialised its barriers
     if (epi) {
         const bool ok = mbar_wait(accf, 0, p.status, 45);
         if (split == 0 && splits > static_cast<uint32_t>(C::EARLY_SPLITS) && warp == 3 && lane == 0)
@@ -1448,7 +1450,9 @@ __global__ void __launch_bounds__(RowqCfg<KIND>::THREADS, 1)
                 packed[i] = *reinterpret_cast<const uint32_t*>(&b);
             }
             if (p.tma_store) {
-                // every epilogue warp is done reading the partials before the staging tiles reuse them
+                // every epilogue warp is done reading the partials before the staging tiles reuse them;
+                // lanes past the last valid row skipped the waits above, and bar.sync wants whole warps
+                __syncwarp();
                 named_barrier_sync(2, 32 * C::QWARPS);
                 // 32 rows x 32 columns per warp, 64B swizzle (16-byte piece q of row r at q ^ ((r >> 1) & 3))
                 uint8_t* stg = smem + (warp - 3) * C::STG_BYTES;

@@ -195,13 +195,15 @@ def test_linear_one_launch_x_16_byte_aligned(fmt, M, N, K):
 @pytest.mark.parametrize("fmt,rule", [("mxfp4", "ceil"), ("mxfp4", "even"), ("nvfp4", "even"), ("mxfp8", "even"),
                                       ("mxfp8", "ceil")])
 @pytest.mark.parametrize("M,N,K", [(33, 96, 512), (129, 1, 640), (300, 128, 320), (1000, 100, 1024), (257, 17, 5120),
-                                   (4000, 96, 256)])
+                                   (4000, 96, 256), (45, 64, 768)])
 def test_linear_small_n_matches_oracle(fmt, rule, M, N, K):
     """More than 32 tokens and N <= 128: mxq_linear is one launch, the small-N kernel quantizing each
     128-row activation tile on its way into the tensor cores (K split over a cluster).  Checked
     against the oracle from the bf16 inputs, fp32 and bf16 out, with ragged M tiles, N = 1 and
     N < 128 column tails, a K tail that leaves the last stage partly empty (K = 320) and one K
-    stage only (K = 256 for FP4: no split)."""
+    stage only (K = 256 for FP4: no split).  Clusters of 2 and 3 CTAs share the reduction by
+    32-row sub-partition; (45, 64, 768) splits K three ways over a tile whose last two
+    sub-partitions hold no valid row, so one CTA receives and stores nothing."""
     if fmt == "mxfp8" and K % 32:
         pytest.skip("K")
     assert mxq.linear_kernel_count(M, N, K, fmt) == 1
