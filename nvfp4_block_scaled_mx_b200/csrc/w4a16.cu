@@ -1056,7 +1056,11 @@ int w16_splits(int64_t tiles, int64_t k_stages, int max_splits) {
     int64_t s = sm_count() / (tiles > 0 ? tiles : 1);
     if (s > max_splits) s = max_splits;
     if (s > k_stages / 2) s = k_stages / 2;
-    return s < 2 ? 1 : static_cast<int>(s);
+    if (s < 2) return 1;
+    // the kernel gives each split ceil(k_stages / s) stages: drop splits that would get none
+    // (9 stages over 4 would leave the last one empty)
+    const int64_t per = ceil_div(k_stages, s);
+    return static_cast<int>(ceil_div(k_stages, per));
 }
 
 template <int FMT, bool F32>

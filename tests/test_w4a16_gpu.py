@@ -36,7 +36,8 @@ def _gpu_w4a16(A, w, N, fmt, out_dtype):
 SHAPES = [(1, 1, 64), (16, 256, 256), (128, 128, 128), (200, 300, 320), (129, 520, 1024), (300, 257, 576),
           (64, 96, 5120), (512, 768, 192), (100, 1000, 2048), (1024, 96, 1024), (777, 1111, 704),
           (32, 19200, 256), (100, 9600, 512),  # these two: more weight tiles than SMs
-          (17, 1024, 4096), (5, 300, 1600)]  # K split over 4 and 3 CTAs at 32 tokens, a ragged last K stage
+          (17, 1024, 4096), (5, 300, 1600),  # K split over 4 and 3 CTAs at 32 tokens, a ragged last K stage
+          (32, 1024, 2304), (48, 512, 2304)]  # 9 K stages: 3 splits of 3 (4 splits would leave one empty)
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
