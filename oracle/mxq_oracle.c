@@ -33,7 +33,8 @@
  *
  * Parity status: every function here is pinned by the CPU test suite against library decoders
  * (ml_dtypes, torch), exact rational arithmetic or brute force, except the NVFP4 operation order
- * and the MXFP8 scale rule, which are readings (the pages do not fix them).
+ * and the CEIL rule applied to MXFP8, which are readings (the pages do not fix them; MXFP8 under
+ * EVEN is the OCP MX rule that the AutoRound card's section 7 cites).
  *
  * Threads: orc_quantize_mt and orc_gemm_mt split the rows (quantizer) or the output columns (GEMM)
  * into contiguous ranges, one per POSIX thread, each running exactly the single-threaded code on its
