@@ -3,12 +3,16 @@
 Each check is chosen so that a plausible slip in the oracle (wrong rule, dropped sign, swapped
 nibbles, wrong block index, transposed operand, missing global scale) fails at least one test:
   - MX quantize against a construction from library casts (ml_dtypes) and exact exponents;
-  - NVFP4 against numpy fp32 arithmetic plus ml_dtypes casts, and a hand-worked block;
+  - NVFP4 against numpy fp32 arithmetic plus ml_dtypes casts, a hand-worked block, and its
+    order-free definition in exact rational arithmetic (nearest E4M3 scale to amax / (6 g),
+    nearest E2M1 value to x / (dec(s) g)) wherever no rounding midpoint is within reach of the
+    fp32 steps;
   - invariants: all-zero blocks, saturation, idempotence, value bounds;
   - scale layout: bijection, round trip, hand-worked offsets;
   - GEMM: numpy fp64 matmul of library-decoded operands, exact integer products, selection.
 """
 import math
+from fractions import Fraction
 
 import ml_dtypes
 import numpy as np
@@ -362,3 +366,78 @@ def test_nvfp4_every_binade_matches_fp32_library_construction(orc, g):
     codes_ref, sf_ref = _nvfp4_reference(x, g)
     assert np.array_equal(sf, sf_ref)
     assert np.array_equal(_unpack_fp4(q), codes_ref)
+
+
+_E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+_E2M1_MIDPOINTS = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+
+
+def _e4m3_positive_table():
+    """(exact value, code) for every finite non-negative E4M3 code, decoded by ml_dtypes."""
+    codes = np.arange(0x7F, dtype=np.uint8)  # 0x7F is NaN
+    vals = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    return [(Fraction(float(v)), int(c)) for v, c in zip(vals, codes)]
+
+
+def _near(q, points, rel):
+    return any(abs(q - p) <= abs(p) * rel for p in points)
+
+
+@pytest.mark.parametrize("g_kind", ["tensor", "one", "small"])
+def test_nvfp4_exact_rounding_away_from_midpoints(orc, g_kind):
+    """NVFP4 against its order-free definition, in exact rational arithmetic: the block scale is the
+    E4M3 value nearest to amax / (6 g) (saturating at 448), and each element is the E2M1 value
+    nearest to x / (dec(s) g), saturating at 6, with x's sign.  Any fp32 order of those steps moves
+    the quotients by a few fp32 ulps at most, so wherever an exact quotient lies further than 2^-20
+    (relative) from a rounding midpoint the result is fixed whatever the order; the rest are skipped,
+    and must be few.  A wrong block size, a global scale applied the other way, a 6 in place of 448
+    or a swapped nibble all fail here."""
+    x = _adversarial_bf16(16, 512, 77, huge=40.0, bs=16)
+    if g_kind == "tensor":
+        g, _ = orc.global_scale(x)
+    else:
+        g = np.float32(1.0 if g_kind == "one" else 3.7e-6)
+    q, sf = orc.quantize(x, orc.NVFP4, 0, g=float(g))
+    codes = _unpack_fp4(q)
+    gq = Fraction(float(g))
+    table = _e4m3_positive_table()  # index = code
+    e4m3_mid = [(table[i][0] + table[i + 1][0]) / 2 for i in range(len(table) - 1)]
+    e2m1_mid = [Fraction(m) for m in _E2M1_MIDPOINTS]
+    xf = x.float().numpy().astype(np.float64).reshape(16, -1, 16)
+    rel = Fraction(1, 1 << 20)
+    n_blocks = xf.shape[0] * xf.shape[1]
+    zero_blocks = checked_s = checked_q = skipped_q = 0
+    for r in range(xf.shape[0]):
+        for b in range(xf.shape[1]):
+            blk = xf[r, b]
+            amax = Fraction(float(np.abs(blk).max()))
+            u = amax / (6 * gq)
+            s_code = int(sf[r, b])
+            if amax == 0:
+                assert s_code == 0
+                zero_blocks += 1
+            elif u >= 448:
+                assert s_code == 0x7E, (r, b)
+                checked_s += 1
+            elif not _near(u, e4m3_mid, rel):
+                best = min(table, key=lambda vc: abs(vc[0] - u))
+                assert s_code == best[1], (r, b, float(u))
+                checked_s += 1
+            dq = table[s_code][0] * gq
+            for i in range(16):
+                xi = float(blk[i])
+                c = int(codes[r, b * 16 + i])
+                sign = 8 if math.copysign(1.0, xi) < 0 else 0
+                if dq == 0:
+                    assert c == sign, (r, b, i)
+                    checked_q += 1
+                    continue
+                v = abs(Fraction(xi)) / dq
+                if _near(v, e2m1_mid, rel):
+                    skipped_q += 1
+                    continue
+                mag = 7 if v > 5 else min(range(8), key=lambda k: abs(Fraction(_E2M1_VALUES[k]) - v))
+                assert c == (mag | sign), (r, b, i, float(v))
+                checked_q += 1
+    assert zero_blocks + checked_s >= 0.95 * n_blocks
+    assert checked_q >= 0.8 * xf.size and skipped_q <= 0.05 * xf.size
