@@ -9,8 +9,10 @@ unchanged copy, which must pass, so the failures come from the planted mistakes 
 The mistakes are the kinds the pins are meant to catch: an off-by-one exponent, a strict instead
 of a non-strict comparison, a wrong clamp, ties rounded away from zero, a wrong saturation value,
 a wrong exponent bias, swapped nibbles, a swizzle that is not a bijection, a dropped global scale,
-a dropped term of a sum, a global scale applied the wrong way, a short block and a wrong global
-scale constant.  Every planted change keeps all memory accesses inside their buffers.
+a dropped term of a sum, a global scale applied the wrong way, a short block, a wrong global
+scale constant, swapped activation columns in the weight-only GEMM, bf16 rounding by truncation
+and a running maximum that forgets its history.  Every planted change keeps all memory accesses
+inside their buffers.
 """
 import importlib.util
 import os
@@ -18,8 +20,10 @@ import shutil
 
 import pytest
 
+import test_oracle_fakequant as FQ
 import test_oracle_formats as F
 import test_oracle_quant as Q
+import test_oracle_w4a16 as W
 
 ORACLE_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle")
 
@@ -77,6 +81,30 @@ MUTANTS = {
         "    volatile float g = amax / 2688.0f;\n",
         "    volatile float g = amax / 448.0f;\n",
         ["nvfp4_library"]),
+    "w4a16_drops_global_scale": (
+        "    double alpha = fmt == ORC_NVFP4 ? gB : 1.0;\n",
+        "    double alpha = 1.0;\n",
+        ["w4a16_nvfp4"]),
+    "w4a16_swaps_activation_columns": (
+        "        for (int64_t k = 0; k < K; k++) arow[i * K + k] = orc_bf16_value(A[m * K + k]);\n",
+        "        for (int64_t k = 0; k < K; k++) arow[i * K + k] = orc_bf16_value(A[m * K + (k ^ 1)]);\n",
+        ["w4a16_mxfp4", "w4a16_exact"]),
+    "bf16_rounding_truncates": (
+        "    uint32_t r = u + 0x7FFFu + ((u >> 16) & 1u);\n",
+        "    uint32_t r = u;\n",
+        ["f32_to_bf16"]),
+    "fake_quant_nibbles_swapped": (
+        "                uint8_t byte = q[(r * K + k) / 2];\n                elem = orc_e2m1_value(k % 2 == 0 ",
+        "                uint8_t byte = q[(r * K + k) / 2];\n                elem = orc_e2m1_value(k % 2 == 1 ",
+        ["fake_quant_mxfp4"]),
+    "fake_quant_nvfp4_drops_global_scale": (
+        "                volatile float d = (float)orc_e4m3_value(s) * g;\n",
+        "                volatile float d = (float)orc_e4m3_value(s);\n",
+        ["fake_quant_nvfp4"]),
+    "running_max_forgets_history": (
+        "    *amax_out = a > amax_in ? a : amax_in;\n",
+        "    *amax_out = a;\n",
+        ["running_max"]),
 }
 
 PINS = {
@@ -96,6 +124,14 @@ PINS = {
     "gemm_exact": lambda o: Q.test_gemm_exact_integers(o),
     "nvfp4_exact": lambda o: [Q.test_nvfp4_exact_rounding_away_from_midpoints(o, k) for k in ("tensor", "one")],
     "nvfp4_library": lambda o: Q.test_nvfp4_matches_fp32_library_construction(o),
+    "w4a16_mxfp4": lambda o: W.test_w4a16_matches_numpy_fp64(o, "mxfp4"),
+    "w4a16_nvfp4": lambda o: W.test_w4a16_matches_numpy_fp64(o, "nvfp4"),
+    "w4a16_exact": lambda o: W.test_w4a16_exact_integers(o),
+    "f32_to_bf16": lambda o: FQ.test_f32_to_bf16_matches_torch(o),
+    "fake_quant_mxfp4": lambda o: FQ.test_fake_quantize_equals_dequantized_codes(o, "mxfp4", "even"),
+    "fake_quant_nvfp4": lambda o: [FQ.test_nvfp4_fake_quantize_is_fp32_product_then_bf16(o, g)
+                                   for g in (1.0 / 2688, 1.0, 3.7e-6)],
+    "running_max": lambda o: FQ.test_running_max_oracle(o),
 }
 
 
