@@ -10,8 +10,9 @@ The mistakes are the kinds the pins are meant to catch: an off-by-one exponent, 
 of a non-strict comparison, a wrong clamp, ties rounded away from zero, a wrong saturation value,
 a wrong exponent bias, swapped nibbles, a swizzle that is not a bijection, a dropped global scale,
 a dropped term of a sum, a global scale applied the wrong way, a short block, a wrong global
-scale constant, swapped activation columns in the weight-only GEMM, bf16 rounding by truncation
-and a running maximum that forgets its history.  Every planted change keeps all memory accesses
+scale constant, swapped activation columns in the weight-only GEMM, bf16 rounding by truncation,
+a running maximum that forgets its history, MX elements scaled one binade off, a wrong E8M0 bias
+and a dropped sign.  Every planted change keeps all memory accesses
 inside their buffers.
 """
 import importlib.util
@@ -101,6 +102,18 @@ MUTANTS = {
         "                volatile float d = (float)orc_e4m3_value(s) * g;\n",
         "                volatile float d = (float)orc_e4m3_value(s);\n",
         ["fake_quant_nvfp4"]),
+    "mx_elements_scaled_one_binade_off": (
+        "                    double v = ldexp(orc_bf16_value(xb[i]), -e); /* exact */\n",
+        "                    double v = ldexp(orc_bf16_value(xb[i]), -e - 1);\n",
+        ["mx_quantize_mxfp4", "mx_quantize_mxfp8"]),
+    "mx_scale_byte_bias": (
+        "                sf[r * kb + b] = (uint8_t)(e + 127);\n",
+        "                sf[r * kb + b] = (uint8_t)(e + 128);\n",
+        ["mx_quantize_mxfp4", "zero_blocks"]),
+    "mx_sign_dropped": (
+        "    unsigned sign = signbit(v) ? 1u : 0u;\n",
+        "    unsigned sign = 0u;\n",
+        ["e2m1_encode_library", "zero_blocks"]),
     "running_max_forgets_history": (
         "    *amax_out = a > amax_in ? a : amax_in;\n",
         "    *amax_out = a;\n",
@@ -132,6 +145,11 @@ PINS = {
     "fake_quant_nvfp4": lambda o: [FQ.test_nvfp4_fake_quantize_is_fp32_product_then_bf16(o, g)
                                    for g in (1.0 / 2688, 1.0, 3.7e-6)],
     "running_max": lambda o: FQ.test_running_max_oracle(o),
+    "mx_quantize_mxfp4": lambda o: [Q.test_mx_quantize_matches_library_construction(o, "mxfp4", r)
+                                    for r in ("even", "ceil")],
+    "mx_quantize_mxfp8": lambda o: [Q.test_mx_quantize_matches_library_construction(o, "mxfp8", r)
+                                    for r in ("even", "ceil")],
+    "zero_blocks": lambda o: Q.test_zero_blocks(o),
 }
 
 
